@@ -1,0 +1,199 @@
+/*
+ * ssmscan.h -- C ABI of libssmscan, a CUDA (sm_100a) implementation of the
+ * Mamba selective-scan forward pass, its single-token decode step and the
+ * Mamba-2 scalar-decay (SSD) chunked scan.
+ *
+ * Definitions (page titles as printed on the source pages):
+ *  - "Mamba状态空间模型的硬件感知推理优化" (ybb.press), section 1:
+ *      h_t = A h_{t-1} + B x_t,   y_t = C h_t;
+ *    section 3.1 (fused scan kernel): y = C h + D x, with the decay
+ *    A_t = exp(A * softplus(dt)) applied per step.
+ *  - "Mamba ... 并行扫描" (mhpq.cn), sections 2.2-2.3 and 3.1: A_d =
+ *    exp(A dt) with A diagonal, so the decay is an elementwise exp; the
+ *    recurrence is evaluated with the combine operator
+ *    (A1, B1) (+) (A2, B2) = (A2 A1, A2 B1 + B2).
+ *  - "从硬件感知到算法革命：Mamba如何重塑序列建模的计算效率"
+ *    (tencentcloud), section 2: dt = softplus(.), B and C depend on the
+ *    input; section 3: the SiLU gate fused after the SSM.
+ *  - "Mamba与选择性SSM" (mlqm.cn), section 5.4: incremental decoding keeps
+ *    only the fixed-size state.
+ *  - "Mamba状态空间模型的硬件感知推理优化" (ybb.press), section 4: the
+ *    Mamba-2 scalar decay h_t = a_t h_{t-1} + b_t x_t, evaluated as a
+ *    parallel/serial hybrid over chunks.
+ *
+ * Per channel (b, d) and state n the selective scan computes
+ *   dt'     = softplus(delta[b,d,t] + delta_bias[d])   (or the sum itself
+ *             when delta_softplus == 0)
+ *   dA      = exp(dt' * A[d,n])
+ *   h[n]    = dA * h[n] + dt' * B[b,n,t] * u[b,d,t]
+ *   y[b,d,t]= (sum_n C[b,n,t] h[n] + D[d] u[b,d,t]) * silu(z[b,d,t])
+ * and returns the final state h_L.  The skip term sits inside the gate.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates no device memory; scratch is passed as `workspace`
+ *    of the size the matching *_workspace_size call reports.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).
+ *    Argument checks run on the host before any launch and return
+ *    synchronously; a failed launch returns SSM_ERR_CUDA.
+ *  - Outputs must not alias inputs, except `state` of ssm_scan_step.
+ *  - Floating-point work is done in fp32; bf16 tensors are widened on load
+ *    and y is rounded to nearest-even on store.  The state and h0 / h_last
+ *    are always fp32.
+ */
+#ifndef SSMSCAN_H
+#define SSMSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ssm_stream_t; /* the same type as cudaStream_t */
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+typedef enum {
+  SSM_OK = 0,
+  SSM_ERR_INVALID_ARG = 1,  /* null required pointer, negative size, bad flag */
+  SSM_ERR_UNSUPPORTED = 2,  /* size or option outside what is implemented  */
+  SSM_ERR_ALIGNMENT = 3,    /* a pointer or stride breaks a required alignment */
+  SSM_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed          */
+  SSM_ERR_WORKSPACE = 5     /* workspace missing or smaller than required    */
+} ssm_status_t;
+
+/* ------------------------------------------------------------------------
+ * Mamba-1 selective scan over a whole sequence.
+ *
+ * Layout (element strides; a stride of 0 selects the contiguous default):
+ *   u, delta, z, y : (batch, dim, seqlen), unit stride along seqlen;
+ *                    *_stride[0] = batch stride, *_stride[1] = dim stride
+ *                    (defaults dim*seqlen and seqlen).
+ *   B, C           : (batch, dstate, seqlen), unit stride along seqlen;
+ *                    *_stride[0] = batch stride, *_stride[1] = state stride
+ *                    (defaults dstate*seqlen and seqlen).
+ *   A              : (dim, dstate) fp32, contiguous.
+ *   D, delta_bias  : (dim) fp32, or NULL (no skip term / zero bias).
+ *   z              : or NULL (no gate).
+ *   h0, h_last     : (batch, dim, dstate) fp32, contiguous; h0 NULL means a
+ *                    zero initial state, h_last NULL means it is not written.
+ * Sizes: batch, dim >= 0; 1 <= dstate <= 16; seqlen >= 0.  seqlen == 0 only
+ * writes h_last (= h0, or zeros).
+ * Element type: `dtype` applies to u, delta, z, B, C and y.
+ * Alignment: every pointer must be aligned to its element size.  Rows that
+ * start on 16-byte boundaries (pointers and strides) take the vectorised
+ * load path; others take a scalar-load path with the same results.
+ * Split-and-resume: scanning [0, m) with h_last = h_m and then [m, L) with
+ * h0 = h_m gives the same y and h_L as one scan (strides allow passing the
+ * two halves of one tensor in place).
+ */
+typedef struct {
+  int64_t batch, dim, dstate, seqlen;
+  ssm_dtype_t dtype;
+  const void* u;
+  const void* delta;
+  const float* A;
+  const void* B;
+  const void* C;
+  const float* D;
+  const void* z;
+  const float* delta_bias;
+  int delta_softplus;
+  const float* h0;
+  void* y;
+  float* h_last;
+  int64_t u_stride[2], delta_stride[2], z_stride[2], y_stride[2];
+  int64_t B_stride[2], C_stride[2];
+} ssm_scan_args_t;
+
+/* Bytes of scratch ssm_scan_fwd needs for these arguments (0 when the whole
+ * sequence runs as one segment).  Only sizes, dtype, strides and pointer
+ * alignment are looked at; null pointers are accepted.  Returns (size_t)-1
+ * for invalid arguments. */
+size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args);
+
+/* Runs the selective scan.  `workspace` (device memory, 16-byte aligned,
+ * at least ssm_scan_fwd_workspace_size bytes, contents ignored and
+ * overwritten) holds the per-segment carries when the sequence is split
+ * across thread blocks; it may be NULL when the size is 0.  The workspace
+ * must not be shared by calls that may overlap on the GPU. */
+ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t workspace_bytes,
+                          ssm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * One decode step ("Mamba与选择性SSM", section 5.4): the scan above for a
+ * single time step, with the state read and overwritten in place.
+ *   u, delta, z, y : (batch, dim) contiguous, `dtype`;
+ *   B, C           : (batch, dstate) contiguous, `dtype`;
+ *   A              : (dim, dstate) fp32;  D, delta_bias : (dim) fp32 or NULL;
+ *   state          : (batch, dim, dstate) fp32, read then written.
+ * Applying it L times reproduces ssm_scan_fwd on the same L steps.
+ * Sizes: 1 <= dstate <= 16.  Needs no workspace. */
+typedef struct {
+  int64_t batch, dim, dstate;
+  ssm_dtype_t dtype;
+  const void* u;
+  const void* delta;
+  const void* z;
+  const void* B;
+  const void* C;
+  const float* A;
+  const float* D;
+  const float* delta_bias;
+  int delta_softplus;
+  float* state;
+  void* y;
+} ssm_step_args_t;
+
+ssm_status_t ssm_scan_step(const ssm_step_args_t* args, ssm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Mamba-2 scalar-decay scan, chunked ("Mamba状态空间模型的硬件感知推理优化",
+ * section 4; chunked hybrid scan, section 4 end and section 5).  Per batch
+ * b and head h with state S (headdim x dstate):
+ *   dt'  = softplus(delta[b,t,h] + delta_bias[h]),  a_t = exp(dt' A[h])
+ *   S    = a_t S + dt' x[b,t,h,:]^T B[b,t,:]
+ *   y[b,t,h,:] = (S C[b,t,:] + D[h] x[b,t,h,:]) * silu(z[b,t,h,:])
+ * Layout (contiguous):
+ *   x, z, y     : (batch, seqlen, nheads, headdim)   `dtype`
+ *   delta       : (batch, seqlen, nheads)            `dtype`
+ *   B, C        : (batch, seqlen, dstate)            `dtype` (shared by all heads)
+ *   A, D, delta_bias : (nheads) fp32 (D, delta_bias may be NULL)
+ *   h0, h_last  : (batch, nheads, headdim, dstate) fp32 or NULL.
+ * chunk is the length of the intra-chunk quadratic block. */
+typedef struct {
+  int64_t batch, seqlen, nheads, headdim, dstate, chunk;
+  ssm_dtype_t dtype;
+  const void* x;
+  const void* delta;
+  const float* A;
+  const void* B;
+  const void* C;
+  const float* D;
+  const float* delta_bias;
+  int delta_softplus;
+  const void* z;
+  const float* h0;
+  void* y;
+  float* h_last;
+} ssm_ssd_args_t;
+
+size_t ssm_scan_fwd_chunked_workspace_size(const ssm_ssd_args_t* args);
+ssm_status_t ssm_scan_fwd_chunked(const ssm_ssd_args_t* args, void* workspace,
+                                  size_t workspace_bytes, ssm_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+const char* ssm_status_string(ssm_status_t status);
+int ssm_version(void); /* major * 10000 + minor * 100 + patch */
+
+/* Description of the CUDA error behind the last SSM_ERR_CUDA returned on the
+ * calling host thread ("" if none).  The string stays valid until the next
+ * failing call on that thread. */
+const char* ssm_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSMSCAN_H */

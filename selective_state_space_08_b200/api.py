@@ -1,0 +1,152 @@
+"""Python binding of libssmscan over torch CUDA tensors.
+
+Argument marshalling only: the functions check devices, dtypes and layouts,
+allocate outputs (and scratch) with torch when the caller passes none, and
+call the C ABI on the current torch stream.  Every step of the computation
+runs in the library's CUDA kernels; nothing here computes.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+
+_DT = {torch.float32: _abi.SSM_F32, torch.bfloat16: _abi.SSM_BF16}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(name, t, dtype=None, dims=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if dims is not None and t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dimensions")
+    return t
+
+
+def _seq_strides(name, t):
+    """(batch stride, row stride) of a (batch, rows, L) tensor with unit stride along L."""
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous along the sequence")
+    return (t.stride(0), t.stride(1))
+
+
+def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last):
+    dt = u.dtype
+    if dt not in _DT:
+        raise ValueError("u must be float32 or bfloat16")
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    for name, t in (("delta", delta), ("z", z), ("y", y)):
+        if t is not None and (t.dtype != dt or tuple(t.shape) != (batch, dim, L)):
+            raise ValueError(f"{name} must be {dt} of shape {(batch, dim, L)}")
+    for name, t in (("B", B), ("C", C)):
+        if t.dtype != dt or tuple(t.shape) != (batch, N, L):
+            raise ValueError(f"{name} must be {dt} of shape {(batch, N, L)}")
+    for name, t, shape in (("A", A, (dim, N)), ("D", D, (dim,)), ("delta_bias", delta_bias, (dim,)),
+                           ("h0", h0, (batch, dim, N)), ("h_last", h_last, (batch, dim, N))):
+        if t is not None:
+            _cuda(name, t, torch.float32)
+            if tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous float32 of shape {shape}")
+    a = _abi.ScanArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = batch, dim, N, L
+    a.dtype = _DT[dt]
+    a.u, a.delta, a.A, a.B, a.C = _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C)
+    a.D, a.z, a.delta_bias = _ptr(D), _ptr(z), _ptr(delta_bias)
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.h0, a.y, a.h_last = _ptr(h0), _ptr(y), _ptr(h_last)
+    for field, name, t in (("u_stride", "u", u), ("delta_stride", "delta", delta), ("z_stride", "z", z),
+                           ("y_stride", "y", y), ("B_stride", "B", B), ("C_stride", "C", C)):
+        if t is not None:
+            sb, sr = _seq_strides(name, t)
+            getattr(a, field)[0] = sb
+            getattr(a, field)[1] = sr
+    return a
+
+
+def scan_fwd_workspace_size(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                            delta_softplus=True, h0=None) -> int:
+    """Bytes of scratch ``scan_fwd`` needs for these tensors."""
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, None, None)
+    n = _abi.load().ssm_scan_fwd_workspace_size(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    return int(n)
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True, h0=None,
+             *, y=None, h_last=None, return_last_state=True, workspace=None, stream=None):
+    """Selective scan (Mamba-1 forward) on CUDA tensors.
+
+    u, delta, z: (batch, dim, L) float32 or bfloat16, unit stride along L;
+    B, C: (batch, N, L) same dtype; A: (dim, N) float32; D, delta_bias: (dim,)
+    float32; h0: (batch, dim, N) float32.  Returns (y, h_last)."""
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+        _cuda(name, t)
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, L)")
+    if y is None:
+        y = torch.empty(u.shape, dtype=u.dtype, device=u.device)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((u.shape[0], u.shape[1], A.shape[1]), dtype=torch.float32,
+                             device=u.device)
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last)
+    lib = _abi.load()
+    need = lib.ssm_scan_fwd_workspace_size(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(int(need), dtype=torch.uint8, device=u.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _abi.check(lib.ssm_scan_fwd(ctypes.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
+               "ssm_scan_fwd")
+    return y, h_last
+
+
+def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+              *, y=None, stream=None):
+    """One decode step; ``state`` (batch, dim, N) float32 is updated in place.
+    u, delta, z: (batch, dim); B, C: (batch, N).  Returns y (batch, dim)."""
+    for name, t in (("state", state), ("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C),
+                    ("D", D), ("z", z), ("delta_bias", delta_bias), ("y", y)):
+        _cuda(name, t)
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if u.dtype not in _DT:
+        raise ValueError("u must be float32 or bfloat16")
+    batch, dim = u.shape
+    N = A.shape[1]
+    if state.dtype != torch.float32 or tuple(state.shape) != (batch, dim, N):
+        raise ValueError("state must be float32 (batch, dim, N)")
+    for name, t, shape, dtype in (("delta", delta, (batch, dim), u.dtype),
+                                  ("z", z, (batch, dim), u.dtype), ("B", B, (batch, N), u.dtype),
+                                  ("C", C, (batch, N), u.dtype), ("A", A, (dim, N), torch.float32),
+                                  ("D", D, (dim,), torch.float32),
+                                  ("delta_bias", delta_bias, (dim,), torch.float32)):
+        if t is not None and (tuple(t.shape) != shape or t.dtype != dtype):
+            raise ValueError(f"{name} must be {dtype} of shape {shape}")
+    if y is None:
+        y = torch.empty((batch, dim), dtype=u.dtype, device=u.device)
+    a = _abi.StepArgs()
+    a.batch, a.dim, a.dstate, a.dtype = batch, dim, N, _DT[u.dtype]
+    a.u, a.delta, a.z, a.B, a.C = _ptr(u), _ptr(delta), _ptr(z), _ptr(B), _ptr(C)
+    a.A, a.D, a.delta_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
+    a.delta_softplus = 1 if delta_softplus else 0
+    a.state, a.y = _ptr(state), _ptr(y)
+    _abi.check(_abi.load().ssm_scan_step(ctypes.byref(a), _stream(stream)), "ssm_scan_step")
+    return y

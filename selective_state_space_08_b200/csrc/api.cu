@@ -1,0 +1,324 @@
+// api.cu -- host side of the libssmscan C ABI: argument checks, work planning
+// and kernel dispatch.  Every entry point is declared in include/ssmscan.h.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdio>
+#include <cstdint>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/ssmscan.h"
+#include "scan_fwd.cuh"
+#include "scan_step.cuh"
+
+namespace {
+
+using namespace ssm;
+
+constexpr int kMaxDevices = 64;
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int device_sm_count() {
+  static int counts[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per
+// (kernel, device).  The cache is keyed by the kernel's address: every
+// kernel template instance has the same function type.
+cudaError_t set_smem(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess) done.insert({kernel, dev});
+  return e;
+}
+
+size_t elem_size(ssm_dtype_t t) { return t == SSM_BF16 ? 2 : 4; }
+
+thread_local char g_last_error[256] = "";
+
+// Maps a CUDA result to a status, remembering the message of a failure.
+ssm_status_t cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return SSM_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorString(e),
+           cudaGetErrorName(e));
+  return SSM_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Mamba-1 selective scan
+// ---------------------------------------------------------------------------
+struct ScanPlan {
+  ScanParams p;
+  bool vec;
+  size_t ws_bytes;
+};
+
+// check_ptrs = false skips the null-pointer checks (workspace-size queries
+// look only at sizes, types and layout).
+ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* out, bool check_ptrs = true) {
+  if (a == nullptr) return SSM_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->dim < 0 || a->seqlen < 0) return SSM_ERR_INVALID_ARG;
+  if (a->dtype != SSM_F32 && a->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+  if (a->dstate < 1 || a->dstate > fwd::kMaxN) return SSM_ERR_UNSUPPORTED;
+  if (a->batch > 65535) return SSM_ERR_UNSUPPORTED;
+  const int64_t L = a->seqlen;
+  const size_t es = elem_size(a->dtype);
+  const bool any_work = a->batch > 0 && a->dim > 0;
+  if (any_work && check_ptrs) {
+    if (a->A == nullptr) return SSM_ERR_INVALID_ARG;
+    if (L > 0 && (a->u == nullptr || a->delta == nullptr || a->B == nullptr ||
+                  a->C == nullptr || a->y == nullptr))
+      return SSM_ERR_INVALID_ARG;
+  }
+  const void* tensors[] = {a->u, a->delta, a->B, a->C, a->z, a->y};
+  for (const void* t : tensors)
+    if (t != nullptr && !aligned(t, es)) return SSM_ERR_ALIGNMENT;
+  const void* f32s[] = {a->A, a->D, a->delta_bias, a->h0, a->h_last};
+  for (const void* t : f32s)
+    if (t != nullptr && !aligned(t, 4)) return SSM_ERR_ALIGNMENT;
+
+  ScanParams& p = out->p;
+  p.batch = a->batch;
+  p.dim = a->dim;
+  p.dstate = a->dstate;
+  p.seqlen = L;
+  p.u = a->u;
+  p.delta = a->delta;
+  p.z = a->z;
+  p.y = a->y;
+  p.B = a->B;
+  p.C = a->C;
+  auto pick = [](int64_t s, int64_t def) { return s == 0 ? def : s; };
+  const int64_t xb = a->dim * L, xd = L, bcb = a->dstate * L, bcn = L;
+  p.u_sb = pick(a->u_stride[0], xb);
+  p.u_sd = pick(a->u_stride[1], xd);
+  p.dl_sb = pick(a->delta_stride[0], xb);
+  p.dl_sd = pick(a->delta_stride[1], xd);
+  p.z_sb = pick(a->z_stride[0], xb);
+  p.z_sd = pick(a->z_stride[1], xd);
+  p.y_sb = pick(a->y_stride[0], xb);
+  p.y_sd = pick(a->y_stride[1], xd);
+  p.B_sb = pick(a->B_stride[0], bcb);
+  p.B_sn = pick(a->B_stride[1], bcn);
+  p.C_sb = pick(a->C_stride[0], bcb);
+  p.C_sn = pick(a->C_stride[1], bcn);
+  const int64_t strides[] = {p.u_sb, p.u_sd, p.dl_sb, p.dl_sd, p.z_sb, p.z_sd,
+                             p.y_sb, p.y_sd, p.B_sb, p.B_sn, p.C_sb, p.C_sn};
+  for (int64_t s : strides)
+    if (s < 0) return SSM_ERR_INVALID_ARG;
+  p.A = a->A;
+  p.D = a->D;
+  p.bias = a->delta_bias;
+  p.softplus = a->delta_softplus ? 1 : 0;
+  p.h0 = a->h0;
+  p.h_last = a->h_last;
+
+  // 16-byte rows take the cp.async path.
+  bool vec = true;
+  for (const void* t : tensors)
+    if (t != nullptr && !aligned(t, 16)) vec = false;
+  const int64_t need = 16 / static_cast<int64_t>(es);
+  for (int64_t s : strides)
+    if (s % need != 0) vec = false;
+  out->vec = vec;
+
+  // L-segments: split the sequence when the channels alone leave the GPU idle.
+  const int64_t ctas = ((a->dim + fwd::kCH - 1) / fwd::kCH) * a->batch;
+  const int64_t sms = device_sm_count();
+  const int64_t target = sms * 8;
+  int64_t nseg = 1;
+  if (any_work && L > 0 && ctas > 0 && ctas < 2 * sms) {
+    const int64_t max_seg = (L + fwd::kTL - 1) / fwd::kTL;
+    nseg = (target + ctas - 1) / ctas;
+    if (nseg > max_seg) nseg = max_seg;
+    if (nseg > 65535) nseg = 65535;
+  }
+  int64_t seg_len = L;
+  if (nseg > 1) {
+    seg_len = (L + nseg - 1) / nseg;
+    seg_len = (seg_len + fwd::kTL - 1) / fwd::kTL * fwd::kTL;
+    nseg = (L + seg_len - 1) / seg_len;
+  }
+  if (seg_len <= 0) seg_len = 1;
+  p.nseg = nseg;
+  p.seg_len = seg_len;
+  out->ws_bytes = nseg > 1 ? static_cast<size_t>(nseg - 1) * a->batch * a->dim *
+                                 (fwd::kMaxN + 1) * sizeof(float)
+                           : 0;
+  return SSM_OK;
+}
+
+template <typename T, int MODE, bool HAS_Z, bool VEC>
+ssm_status_t launch_fwd(const ScanParams& p, cudaStream_t stream) {
+  auto kernel = fwd::scan_fwd_kernel<T, MODE, HAS_Z, VEC>;
+  const size_t smem = sizeof(fwd::Smem<T>);
+  ssm_status_t st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem),
+                                "scan_fwd: shared-memory opt-in");
+  if (st != SSM_OK) return st;
+  const dim3 grid(static_cast<unsigned>((p.dim + fwd::kCH - 1) / fwd::kCH),
+                  static_cast<unsigned>(p.batch),
+                  static_cast<unsigned>(MODE == fwd::kAgg ? p.nseg - 1 : p.nseg));
+  kernel<<<grid, fwd::kThreads, smem, stream>>>(p);
+  return cuda_status(cudaGetLastError(), MODE == fwd::kAgg ? "scan_fwd: aggregate pass launch"
+                                                           : "scan_fwd: scan pass launch");
+}
+
+template <typename T, bool VEC>
+ssm_status_t run_fwd(const ScanParams& p, cudaStream_t stream) {
+  ssm_status_t st = SSM_OK;
+  if (p.nseg > 1) {
+    st = launch_fwd<T, fwd::kAgg, false, VEC>(p, stream);
+    if (st != SSM_OK) return st;
+    const int64_t total = p.batch * p.dim * fwd::kMaxN;
+    const int threads = 256;
+    fwd::scan_carry_kernel<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0,
+                             stream>>>(p);
+    st = cuda_status(cudaGetLastError(), "scan_fwd: carry launch");
+    if (st != SSM_OK) return st;
+  }
+  return p.z != nullptr ? launch_fwd<T, fwd::kFull, true, VEC>(p, stream)
+                        : launch_fwd<T, fwd::kFull, false, VEC>(p, stream);
+}
+
+// ---------------------------------------------------------------------------
+// decode step
+// ---------------------------------------------------------------------------
+template <typename T, bool HAS_Z, bool VEC4>
+ssm_status_t launch_step(const StepParams& p, cudaStream_t stream) {
+  const int64_t threads = p.batch * p.dim * step::kNG;
+  const int64_t blocks = (threads + step::kThreads - 1) / step::kThreads;
+  if (blocks > INT_MAX) return SSM_ERR_UNSUPPORTED;
+  step::scan_step_kernel<T, HAS_Z, VEC4>
+      <<<static_cast<unsigned>(blocks), step::kThreads, 0, stream>>>(p);
+  return cuda_status(cudaGetLastError(), "scan_step: launch");
+}
+
+template <typename T>
+ssm_status_t run_step(const StepParams& p, bool vec4, cudaStream_t stream) {
+  if (p.z != nullptr)
+    return vec4 ? launch_step<T, true, true>(p, stream) : launch_step<T, true, false>(p, stream);
+  return vec4 ? launch_step<T, false, true>(p, stream) : launch_step<T, false, false>(p, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args) {
+  ScanPlan plan;
+  if (plan_scan(args, &plan, false) != SSM_OK) return static_cast<size_t>(-1);
+  return plan.ws_bytes;
+}
+
+ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t workspace_bytes,
+                          ssm_stream_t stream_) {
+  ScanPlan plan;
+  ssm_status_t st = plan_scan(args, &plan);
+  if (st != SSM_OK) return st;
+  ScanParams& p = plan.p;
+  if (p.batch == 0 || p.dim == 0) return SSM_OK;
+  if (plan.ws_bytes > 0) {
+    if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return SSM_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return SSM_ERR_ALIGNMENT;
+    float* ws = static_cast<float*>(workspace);
+    const int64_t slots = (p.nseg - 1) * p.batch * p.dim;
+    p.carry_h = ws;
+    p.carry_dt = ws + slots * fwd::kMaxN;
+  } else {
+    p.carry_h = nullptr;
+    p.carry_dt = nullptr;
+  }
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (args->dtype == SSM_BF16)
+    return plan.vec ? run_fwd<__nv_bfloat16, true>(p, stream)
+                    : run_fwd<__nv_bfloat16, false>(p, stream);
+  return plan.vec ? run_fwd<float, true>(p, stream) : run_fwd<float, false>(p, stream);
+}
+
+ssm_status_t ssm_scan_step(const ssm_step_args_t* a, ssm_stream_t stream_) {
+  if (a == nullptr) return SSM_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->dim < 0) return SSM_ERR_INVALID_ARG;
+  if (a->dtype != SSM_F32 && a->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+  if (a->dstate < 1 || a->dstate > step::kNG * step::kNPT) return SSM_ERR_UNSUPPORTED;
+  if (a->batch == 0 || a->dim == 0) return SSM_OK;
+  if (a->u == nullptr || a->delta == nullptr || a->B == nullptr || a->C == nullptr ||
+      a->A == nullptr || a->state == nullptr || a->y == nullptr)
+    return SSM_ERR_INVALID_ARG;
+  const size_t es = elem_size(a->dtype);
+  const void* tensors[] = {a->u, a->delta, a->z, a->B, a->C, a->y};
+  for (const void* t : tensors)
+    if (t != nullptr && !aligned(t, es)) return SSM_ERR_ALIGNMENT;
+  const void* f32s[] = {a->A, a->D, a->delta_bias, a->state};
+  for (const void* t : f32s)
+    if (t != nullptr && !aligned(t, 4)) return SSM_ERR_ALIGNMENT;
+  StepParams p;
+  p.batch = a->batch;
+  p.dim = a->dim;
+  p.dstate = a->dstate;
+  p.u = a->u;
+  p.delta = a->delta;
+  p.z = a->z;
+  p.B = a->B;
+  p.C = a->C;
+  p.A = a->A;
+  p.D = a->D;
+  p.bias = a->delta_bias;
+  p.softplus = a->delta_softplus ? 1 : 0;
+  p.state = a->state;
+  p.y = a->y;
+  const bool vec4 = a->dstate == 16 && aligned(a->state, 16);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  return a->dtype == SSM_BF16 ? run_step<__nv_bfloat16>(p, vec4, stream)
+                              : run_step<float>(p, vec4, stream);
+}
+
+size_t ssm_scan_fwd_chunked_workspace_size(const ssm_ssd_args_t* args) {
+  (void)args;
+  return static_cast<size_t>(-1);
+}
+
+ssm_status_t ssm_scan_fwd_chunked(const ssm_ssd_args_t* args, void* workspace,
+                                  size_t workspace_bytes, ssm_stream_t stream) {
+  (void)args;
+  (void)workspace;
+  (void)workspace_bytes;
+  (void)stream;
+  return SSM_ERR_UNSUPPORTED;
+}
+
+const char* ssm_status_string(ssm_status_t s) {
+  switch (s) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_INVALID_ARG: return "invalid argument";
+    case SSM_ERR_UNSUPPORTED: return "unsupported size or option";
+    case SSM_ERR_ALIGNMENT: return "misaligned pointer or stride";
+    case SSM_ERR_CUDA: return "CUDA error";
+    case SSM_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int ssm_version(void) { return 100; }
+
+const char* ssm_last_error_string(void) { return g_last_error; }
+
+}  // extern "C"

@@ -16,10 +16,10 @@ Distributions (the workload descriptions this library is measured on):
 * D_d ~ N(0, 1);
 * Mamba-2 heads: A_h = -exp(U(ln 1, ln 16)).
 
-Every tensor row comes from its own stream ``default_rng([seed, tensor_id,
-row])``, so any subset of rows can be regenerated on its own: the oracle can
-be run on sampled channels of a workload too large for it, and the rows are
-generated in parallel threads.  bf16 tensors are rounded to nearest-even
+Tensor rows come in blocks of 64, each block from its own stream
+``default_rng([seed, tensor_id, block])``, so any subset of rows can be
+regenerated on its own: the oracle can be run on sampled channels of a
+workload too large for it, and the blocks are generated in parallel threads.  bf16 tensors are rounded to nearest-even
 from the float32 draw; both sides receive exactly those values.
 """
 from __future__ import annotations
@@ -70,24 +70,42 @@ def _stream(seed: int, tensor: int, row: int = 0) -> np.random.Generator:
     return np.random.default_rng([int(seed), int(tensor), int(row)])
 
 
+ROWS_PER_STREAM = 64
+
+
 def normal_rows(seed: int, tensor: int, rows, length: int, dtype: str = "f32",
-                threads: int | None = None) -> np.ndarray:
+                threads: int | None = None, bits: bool = False) -> np.ndarray:
     """N(0,1) rows ``rows`` (iterable of ints) of one tensor, each ``length`` long,
-    rounded to ``dtype``; returned as float32 of shape (len(rows), length)."""
-    rows = list(rows)
-    out = np.empty((len(rows), length), dtype=np.float32)
+    rounded to ``dtype``; returned as float32 of shape (len(rows), length), or,
+    with ``bits`` and dtype "bf16", as the uint16 bfloat16 bit patterns.
 
-    def fill(i):
-        v = _stream(seed, tensor, rows[i]).standard_normal(length, dtype=np.float32)
-        out[i] = round_to(v, dtype)
+    Row r is row r % 64 of the (64, length) block drawn from the stream
+    ``default_rng([seed, tensor, r // 64])``, so a row's values do not depend
+    on which other rows are requested."""
+    rows = [int(r) for r in rows]
+    as_bits = bits and dtype == "bf16"
+    out = np.empty((len(rows), length), dtype=np.uint16 if as_bits else np.float32)
+    blocks: dict[int, list[tuple[int, int]]] = {}
+    for i, r in enumerate(rows):
+        blocks.setdefault(r // ROWS_PER_STREAM, []).append((i, r % ROWS_PER_STREAM))
 
+    def fill(item):
+        blk, members = item
+        need = max(m for _, m in members) + 1
+        v = _stream(seed, tensor, blk).standard_normal((ROWS_PER_STREAM, length),
+                                                        dtype=np.float32)[:need]
+        v = to_bf16_bits(v).reshape(v.shape) if as_bits else round_to(v, dtype)
+        for i, m in members:
+            out[i] = v[m]
+
+    items = list(blocks.items())
     n = threads or min(32, os.cpu_count() or 1)
-    if len(rows) * length < (1 << 20) or n == 1:
-        for i in range(len(rows)):
-            fill(i)
+    if len(items) == 1 or n == 1 or len(rows) * length < (1 << 20):
+        for it in items:
+            fill(it)
     else:
         with ThreadPoolExecutor(n) as ex:
-            list(ex.map(fill, range(len(rows))))
+            list(ex.map(fill, items))
     return out
 
 
@@ -106,7 +124,7 @@ def scan_params(seed: int, dim: int, dstate: int, s_range=(1e-3, 1e-1)):
 
 def make_scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str = "f32",
                      gate: bool = True, seed: int = 0, s_range=(1e-3, 1e-1),
-                     channels=None, h0: bool = False) -> dict:
+                     channels=None, h0: bool = False, bits: bool = False) -> dict:
     """Inputs of one selective scan, as float32 arrays holding values exactly
     representable in ``dtype``.
 
@@ -116,7 +134,8 @@ def make_scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str 
     ``channels`` (a list of (b, d) pairs) restricts u/delta/z/h0 to those
     rows, returned with shape (1, len(channels), seqlen), together with the
     matching A/D/bias rows; B and C are then those of the batch of the
-    channels, which must all share one b.
+    channels, which must all share one b.  With ``bits`` and dtype "bf16" the
+    sequence tensors come back as uint16 bfloat16 bit patterns.
     """
     A, D, bias = scan_params(seed, dim, dstate, s_range)
     if channels is None:
@@ -136,13 +155,16 @@ def make_scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str 
     out = {
         "A": np.ascontiguousarray(A[dsel]), "D": np.ascontiguousarray(D[dsel]),
         "delta_bias": np.ascontiguousarray(bias[dsel]),
-        "u": normal_rows(seed, T_U, rows, seqlen, dtype).reshape(shape),
-        "delta": normal_rows(seed, T_DELTA, rows, seqlen, dtype).reshape(shape),
-        "z": normal_rows(seed, T_Z, rows, seqlen, dtype).reshape(shape) if gate else None,
+        "u": normal_rows(seed, T_U, rows, seqlen, dtype, bits=bits).reshape(shape),
+        "delta": normal_rows(seed, T_DELTA, rows, seqlen, dtype, bits=bits).reshape(shape),
+        "z": (normal_rows(seed, T_Z, rows, seqlen, dtype, bits=bits).reshape(shape)
+              if gate else None),
     }
     bc_rows = [b * dstate + n for b in bsel for n in range(dstate)]
-    out["B"] = normal_rows(seed, T_B, bc_rows, seqlen, dtype).reshape(len(bsel), dstate, seqlen)
-    out["C"] = normal_rows(seed, T_C, bc_rows, seqlen, dtype).reshape(len(bsel), dstate, seqlen)
+    out["B"] = normal_rows(seed, T_B, bc_rows, seqlen, dtype, bits=bits).reshape(
+        len(bsel), dstate, seqlen)
+    out["C"] = normal_rows(seed, T_C, bc_rows, seqlen, dtype, bits=bits).reshape(
+        len(bsel), dstate, seqlen)
     out["h0"] = (normal_rows(seed, T_H0, rows, dstate, "f32").reshape(shape[0], shape[1], dstate)
                  if h0 else None)
     return out

@@ -1,0 +1,106 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from selective_state_space_08_b200 import _abi, build
+
+NULL = None
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = _abi.header_functions()
+    assert set(names) >= {"ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_step",
+                          "ssm_scan_fwd_chunked", "ssm_scan_fwd_chunked_workspace_size",
+                          "ssm_status_string", "ssm_version", "ssm_last_error_string"}
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    for n in names:
+        assert f" T {n}" in out, n
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.ssm_status_string(code)
+    assert lib.ssm_version() >= 100
+
+
+def _args(**kw):
+    a = _abi.ScanArgs()
+    a.batch, a.dim, a.dstate, a.seqlen = 2, 40, 16, 100
+    a.dtype = _abi.SSM_BF16
+    fake = 0x10000  # never dereferenced: every case below fails on the host
+    for f in ("u", "delta", "A", "B", "C", "y"):
+        setattr(a, f, fake)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dstate=0), 2), (dict(dstate=17), 2), (dict(batch=-1), 1), (dict(seqlen=-3), 1),
+    (dict(dtype=7), 1), (dict(u=None), 1), (dict(A=None), 1), (dict(y=None), 1),
+    (dict(u=0x10001), 3), (dict(A=0x10002), 3), (dict(batch=70000), 2),
+])
+def test_scan_fwd_rejects_bad_arguments(lib, kw, status):
+    a = _args(**kw)
+    assert lib.ssm_scan_fwd(ctypes.byref(a), None, 0, None) == status
+
+
+def test_scan_fwd_null_args(lib):
+    assert lib.ssm_scan_fwd(None, None, 0, None) == 1
+    assert lib.ssm_scan_fwd_workspace_size(None) == ctypes.c_size_t(-1).value
+
+
+def test_workspace_required_for_long_sequences(lib):
+    a = _args(batch=1, dim=64, seqlen=1 << 20)
+    need = lib.ssm_scan_fwd_workspace_size(ctypes.byref(a))
+    assert 0 < need < (1 << 30)
+    assert lib.ssm_scan_fwd(ctypes.byref(a), None, 0, None) == 5
+    assert lib.ssm_scan_fwd(ctypes.byref(a), 0x10000, need - 1, None) == 5
+    assert lib.ssm_scan_fwd(ctypes.byref(a), 0x10008, need, None) == 3
+
+
+def test_workspace_query_ignores_pointers(lib):
+    a = _args(batch=1, dim=64, seqlen=1 << 20, u=None, delta=None, A=None, B=None, C=None, y=None)
+    assert 0 < lib.ssm_scan_fwd_workspace_size(ctypes.byref(a)) < (1 << 30)
+
+
+def test_no_workspace_when_channels_fill_the_gpu(lib):
+    a = _args(batch=8, dim=1536, seqlen=2048)
+    assert lib.ssm_scan_fwd_workspace_size(ctypes.byref(a)) == 0
+
+
+def test_empty_problems_are_no_ops(lib):
+    a = _args(batch=0)
+    assert lib.ssm_scan_fwd(ctypes.byref(a), None, 0, None) == 0
+    a = _args(dim=0)
+    assert lib.ssm_scan_fwd(ctypes.byref(a), None, 0, None) == 0
+
+
+def test_step_rejects_bad_arguments(lib):
+    s = _abi.StepArgs()
+    s.batch, s.dim, s.dstate, s.dtype = 2, 3, 16, 0
+    assert lib.ssm_scan_step(ctypes.byref(s), None) == 1  # null pointers
+    s.dstate = 17
+    assert lib.ssm_scan_step(ctypes.byref(s), None) == 2
+    assert lib.ssm_scan_step(None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from selective_state_space_08_b200 import api
+    x = torch.zeros(1, 2, 3)
+    with pytest.raises(ValueError):
+        api.scan_fwd(x, x, torch.zeros(2, 4), torch.zeros(1, 4, 3), torch.zeros(1, 4, 3))
