@@ -122,6 +122,32 @@ size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args);
 ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t workspace_bytes,
                           ssm_stream_t stream);
 
+/* Bytes of the library's static device scratch used by ssm_scan_fwd_noalloc. */
+#define SSM_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/* The selective scan for callers that cannot allocate device memory: code
+ * running inside a host framework that owns every device buffer and forbids
+ * allocation while it executes (an inference-engine plugin, for instance),
+ * or code on a latency-critical path that cannot afford cudaMalloc's implicit
+ * synchronisation.  The pages have no counterpart to this entry point: it is
+ * a packaging of ssm_scan_fwd.
+ *
+ * Arguments, layouts and results are those of ssm_scan_fwd; the caller still
+ * passes every input and output.  The scratch that ssm_scan_fwd takes as
+ * `workspace` comes instead from one array of SSM_NOALLOC_SCRATCH_BYTES
+ * (4 MiB) in the library's device memory, which every GPU that loads the
+ * library holds until the process exits.  The call allocates nothing.
+ *  - The first call on a device looks up that array's device address (once
+ *    per device, with that device current); make the first call on each
+ *    device before any stream capture.
+ *  - A call that would need more scratch than the array holds returns
+ *    SSM_ERR_WORKSPACE, and ssm_last_error_string() says how much it needed.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (every call overwrites the part it reads before reading it).  Calls that
+ *    may overlap on the GPU (other streams, other host threads) race on it
+ *    and must be serialised by the caller. */
+ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_args_t* args, ssm_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * One decode step ("Mamba与选择性SSM", section 5.4): the scan above for a
  * single time step, with the state read and overwritten in place.

@@ -118,6 +118,22 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     return y, h_last
 
 
+def scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                     h0=None, *, y, h_last=None, stream=None):
+    """``scan_fwd`` for callers that cannot allocate device memory: ``y`` (and
+    ``h_last`` if wanted) must be passed in, and the scratch comes from the
+    library's static 4 MiB device array (see ssm_scan_fwd_noalloc in
+    include/ssmscan.h: first call on a device before any stream capture;
+    overlapping calls race on the shared array)."""
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+        _cuda(name, t)
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last)
+    _abi.check(_abi.load().ssm_scan_fwd_noalloc(ctypes.byref(a), _stream(stream)),
+               "ssm_scan_fwd_noalloc")
+    return y, h_last
+
+
 def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
               *, y=None, stream=None):
     """One decode step; ``state`` (batch, dim, N) float32 is updated in place.

@@ -219,6 +219,32 @@ ssm_status_t run_step(const StepParams& p, bool vec4, cudaStream_t stream) {
   return vec4 ? launch_step<T, false, true>(p, stream) : launch_step<T, false, false>(p, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Static scratch for ssm_scan_fwd_noalloc.  In host code the name below is a
+// host-side stand-in, not a device address: the address kernels must use is
+// looked up with cudaGetSymbolAddress, once per device.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = SSM_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+cudaError_t noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* ptrs[kMaxDevices] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -252,6 +278,25 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t w
     return plan.vec ? run_fwd<__nv_bfloat16, true>(p, stream)
                     : run_fwd<__nv_bfloat16, false>(p, stream);
   return plan.vec ? run_fwd<float, true>(p, stream) : run_fwd<float, false>(p, stream);
+}
+
+ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_args_t* args, ssm_stream_t stream) {
+  ScanPlan plan;
+  ssm_status_t st = plan_scan(args, &plan);
+  if (st != SSM_OK) return st;
+  if (plan.ws_bytes > kNoAllocScratchBytes) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "ssm_scan_fwd_noalloc: needs %zu bytes of scratch, the static scratch holds %zu",
+             plan.ws_bytes, kNoAllocScratchBytes);
+    return SSM_ERR_WORKSPACE;
+  }
+  if (plan.p.batch == 0 || plan.p.dim == 0) return SSM_OK;
+  void* ws = nullptr;
+  if (plan.ws_bytes > 0) {
+    st = cuda_status(noalloc_scratch(&ws), "ssm_scan_fwd_noalloc: scratch address lookup");
+    if (st != SSM_OK) return st;
+  }
+  return ssm_scan_fwd(args, ws, plan.ws_bytes, stream);
 }
 
 ssm_status_t ssm_scan_step(const ssm_step_args_t* a, ssm_stream_t stream_) {

@@ -21,7 +21,8 @@ def test_library_exports_every_declared_function(lib):
     names = _abi.header_functions()
     assert set(names) >= {"ssm_scan_fwd", "ssm_scan_fwd_workspace_size", "ssm_scan_step",
                           "ssm_scan_fwd_chunked", "ssm_scan_fwd_chunked_workspace_size",
-                          "ssm_status_string", "ssm_version", "ssm_last_error_string"}
+                          "ssm_status_string", "ssm_version", "ssm_last_error_string",
+                          "ssm_scan_fwd_noalloc"}
     for n in names:
         assert hasattr(lib, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
