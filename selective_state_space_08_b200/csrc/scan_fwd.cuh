@@ -5,19 +5,31 @@
 //   dt' = softplus(delta + bias_d);  dA = exp(dt' A[d,n]);
 //   h[n] = dA h[n] + dt' B[b,n,t] u;  y = (sum_n C[b,n,t] h[n] + D_d u) silu(z).
 //
-// Work decomposition.  The scan is done sequentially in time by each thread
-// (the work-optimal form: one multiply-add per state and step), with
-// parallelism over channels and state groups: kNG = 4 lanes share one
-// channel, each owning kNPT = 4 of the (up to) 16 states, so a 128-thread
-// block covers kCH = 32 channels.  Each input element is read from HBM once:
-// tiles of kTL time steps of u / delta / z (kCH rows) and B / C (16 rows)
-// are staged into shared memory with 16-byte cp.async copies, two tiles in
-// flight.  Per tile the block converts B and C to fp32 once (they are shared
-// by every channel of the batch) and computes dt' and dt' * u per element
-// once (shared by the 4 lanes of a channel).  The partial sums C.h of the 4
-// lanes are reduced through shared memory in sub-tiles of 8 steps, after
-// which each lane finishes 2 steps: skip term, gate, rounding to the output
-// type.  y tiles leave through shared memory with 16-byte stores.
+// Work decomposition.  Each thread runs its states sequentially in time (the
+// work-optimal form: one multiply-add per state and step), with parallelism
+// over channels and state groups: kNG = 4 lanes share one channel, each
+// owning kNPT = 4 of the (up to) 16 states as two packed pairs, so a
+// 128-thread block covers kCH = 32 channels.
+//
+// The bound at 16 states is arithmetic, not HBM: per element 16 exponentials
+// and ~70 fp32 lane-operations against 8 bytes.  The special-function unit
+// gives 16 exponentials per SM per clock against 128 FP32 lanes, so part of
+// the decays (kPolySteps of every 8 steps, on one state pair) is evaluated
+// as a polynomial on the FMA pipe (exp2_poly.cuh) to balance the two pipes.
+// The state updates use packed f32x2 instructions, which halve issue slots.
+// All decays of an 8-step sub-tile are computed before its state updates, so
+// the special-function latency overlaps the recurrence.
+//
+// Data movement.  Each input element is read from HBM once: tiles of kTL time
+// steps of u and delta (kCH rows) and of B and C (16 rows) are staged into
+// shared memory with 16-byte cp.async copies; the next tile's copies are in
+// flight during the current tile's scan.  Per tile the block converts B and
+// C to fp32 once (shared by every channel of the batch) and computes dt'
+// (clamped for the decay argument) and dt' u once per element (shared by the
+// 4 lanes of a channel).  The partial sums C.h of the 4 lanes are reduced
+// with a shuffle butterfly per 8-step sub-tile; each lane then finishes 2 steps
+// (skip term, gate, rounding), reading z and writing y straight from and to
+// global memory.
 //
 // Long sequences with few channels are split into L-segments so that the
 // grid fills the GPU (page "Mamba ... 并行扫描", section 2.3: block-local
@@ -30,6 +42,7 @@
 // its incoming state.  No block ever waits on another.
 #pragma once
 #include "common.cuh"
+#include "exp2_poly.cuh"
 
 namespace ssm {
 
@@ -57,31 +70,138 @@ namespace fwd {
 
 constexpr int kThreads = 128;
 constexpr int kNG = 4;                  // lanes per channel
-constexpr int kNPT = 4;                 // states per lane
+constexpr int kNPT = 4;                 // states per lane (two packed pairs)
 constexpr int kMaxN = kNG * kNPT;       // 16
 constexpr int kCH = kThreads / kNG;     // channels per block
 constexpr int kTL = 64;                 // time steps per tile
 constexpr int kSub = 8;                 // steps per reduction sub-tile
+constexpr int kPolySteps = 0;           // per sub-tile: steps whose 2nd pair uses exp2_poly2
 constexpr int kFull = 0, kAgg = 1;
+// |dt' A log2(e)| is clamped to this before the decay exponential: beyond it
+// the decay is below 2^-126 (or the state overflows anyway).
+constexpr float kMaxDecayArg = 126.0f;
 
 template <typename T>
 struct Smem {
   static constexpr int kEPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
   static constexpr int kRow = kTL + kEPC;            // raw row: tile + 16-byte pad
-  T raw_u[2][kCH][kRow];
-  T raw_dl[2][kCH][kRow];
-  T raw_z[2][kCH][kRow];
-  T raw_B[2][kMaxN][kRow];
-  T raw_C[2][kMaxN][kRow];
-  T yout[kCH][kRow];
-  float dtp[kCH][kTL + 4];   // dt' per (channel, step)
+  T raw_u[2][kCH][kRow];     // u is read again by the epilogue: two buffers
+  T raw_dl[kCH][kRow];       // delta, B, C are consumed by the per-tile prep
+  T raw_B[kMaxN][kRow];
+  T raw_C[kMaxN][kRow];
+  float dtp[kCH][kTL + 4];   // dt', clamped, per (channel, step): decay argument
   float du[kCH][kTL + 4];    // dt' * u
-  float Bf[kTL][kMaxN];      // fp32 B, 16-byte chunks swizzled by (t >> 1) & 3
+  float Bf[kTL][kMaxN];      // fp32 B, [step][state]
   float Cf[kTL][kMaxN];
-  float red[kCH][kNG][kSub];  // partial C.h of each lane
 };
 
-__device__ __forceinline__ int bc_swizzle(int t) { return (t >> 1) & 3; }
+// softplus for a pair (see softplus_f in common.cuh for the three ranges; the
+// series threshold here is e^s < 1/16, with 6 terms).
+__device__ __forceinline__ float2 softplus2(float2 s) {
+  const float2 l2e = __fmul2_rn(s, make_float2(kLog2e, kLog2e));
+  const float2 e = make_float2(ex2_approx(l2e.x), ex2_approx(l2e.y));
+  float2 p = __ffma2_rn(e, make_float2(-1.f / 6.f, -1.f / 6.f), make_float2(0.2f, 0.2f));
+  p = __ffma2_rn(p, e, make_float2(-0.25f, -0.25f));
+  p = __ffma2_rn(p, e, make_float2(1.f / 3.f, 1.f / 3.f));
+  p = __ffma2_rn(p, e, make_float2(-0.5f, -0.5f));
+  p = __ffma2_rn(p, e, make_float2(1.f, 1.f));
+  p = __fmul2_rn(p, e);
+  const float2 one_e = __fadd2_rn(e, make_float2(1.f, 1.f));
+  const float2 lg = __fmul2_rn(make_float2(lg2_approx(one_e.x), lg2_approx(one_e.y)),
+                               make_float2(kLn2, kLn2));
+  constexpr float kSeriesMax = -2.7725887f;  // ln(1/16)
+  float2 r;
+  r.x = s.x > 20.f ? s.x : (s.x < kSeriesMax ? p.x : lg.x);
+  r.y = s.y > 20.f ? s.y : (s.y < kSeriesMax ? p.y : lg.y);
+  return r;
+}
+
+// silu for the gate.  bf16 outputs: z sigmoid(z) = z (1 + tanh(z / 2)) / 2 on
+// one MUFU op (its ~5e-4 relative error is below bf16's own rounding of y);
+// fp32 outputs: z / (1 + 2^(-z log2 e)) on two MUFU ops.
+template <typename T>
+__device__ __forceinline__ float gate_silu(float z);
+template <>
+__device__ __forceinline__ float gate_silu<float>(float z) {
+  return silu_f(z);
+}
+template <>
+__device__ __forceinline__ float gate_silu<__nv_bfloat16>(float z) {
+  const float hz = 0.5f * z;
+  return fmaf(hz, tanh_approx(hz), hz);
+}
+
+template <typename T>
+__device__ __forceinline__ float2 load_pair(const T* p);
+template <>
+__device__ __forceinline__ float2 load_pair<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <>
+__device__ __forceinline__ float2 load_pair<float>(const float* p) {
+  return *reinterpret_cast<const float2*>(p);
+}
+template <typename T>
+__device__ __forceinline__ void store_pair(T* p, float a, float b);
+template <>
+__device__ __forceinline__ void store_pair<__nv_bfloat16>(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+template <>
+__device__ __forceinline__ void store_pair<float>(float* p, float a, float b) {
+  *reinterpret_cast<float2*>(p) = make_float2(a, b);
+}
+
+// Two consecutive elements kept in their storage format until used.
+template <typename T>
+struct RawPair;
+template <>
+struct RawPair<__nv_bfloat16> {
+  uint32_t w = 0;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint32_t*>(p); }
+  __device__ __forceinline__ void load_scalar(const __nv_bfloat16* p, bool first, bool second) {
+    const uint32_t lo = first ? static_cast<uint32_t>(__bfloat16_as_ushort(p[0])) : 0u;
+    const uint32_t hi = second ? static_cast<uint32_t>(__bfloat16_as_ushort(p[1])) : 0u;
+    w = lo | (hi << 16);
+  }
+  __device__ __forceinline__ float2 get() const {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+};
+template <>
+struct RawPair<float> {
+  float2 v = make_float2(0.f, 0.f);
+  __device__ __forceinline__ void load(const float* p) { v = *reinterpret_cast<const float2*>(p); }
+  __device__ __forceinline__ void load_scalar(const float* p, bool first, bool second) {
+    v = make_float2(first ? p[0] : 0.f, second ? p[1] : 0.f);
+  }
+  __device__ __forceinline__ float2 get() const { return v; }
+};
+
+// The decays 2^(dt' A log2 e) of one 8-step sub-tile for a lane's two state pairs.
+struct SubDecays {
+  float2 a01[kSub], a23[kSub];
+};
+
+__device__ __forceinline__ void sub_decays(const float* dtp_row, float2 A01, float2 A23,
+                                           SubDecays& out) {
+  float dts[kSub];
+  *reinterpret_cast<float4*>(&dts[0]) = *reinterpret_cast<const float4*>(dtp_row);
+  *reinterpret_cast<float4*>(&dts[4]) = *reinterpret_cast<const float4*>(dtp_row + 4);
+#pragma unroll
+  for (int tt = 0; tt < kSub; ++tt) {
+    const float2 dt2 = make_float2(dts[tt], dts[tt]);
+    const float2 x01 = __fmul2_rn(dt2, A01);
+    out.a01[tt] = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+    if (tt < kPolySteps) {
+      out.a23[tt] = exp2_poly2(dt2, A23);
+    } else {
+      const float2 x23 = __fmul2_rn(dt2, A23);
+      out.a23[tt] = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+    }
+  }
+}
 
 template <typename T, int MODE, bool HAS_Z, bool VEC>
 __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) {
@@ -106,60 +226,62 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
 
   const T* gu = static_cast<const T*>(p.u);
   const T* gdl = static_cast<const T*>(p.delta);
-  const T* gz = static_cast<const T*>(p.z);
   const T* gB = static_cast<const T*>(p.B);
   const T* gC = static_cast<const T*>(p.C);
 
   // ---- per-thread constants and incoming state -------------------------------
-  float A2[kNPT], h[kNPT];
+  float A2[kNPT], hin[kNPT];
+  float amax = 0.f;
 #pragma unroll
   for (int k = 0; k < kNPT; ++k) {
     const int n = g * kNPT + k;
     const bool ok = ch_ok && n < N;
     A2[k] = ok ? p.A[d * N + n] * kLog2e : 0.f;
-    float hin = 0.f;
+    amax = fmaxf(amax, fabsf(A2[k]));
+    float v = 0.f;
     if (MODE == kFull && ok) {
-      if (seg == 0) {
-        hin = p.h0 ? p.h0[bd * N + n] : 0.f;
-      } else {
-        hin = p.carry_h[((seg - 1) * p.batch * p.dim + bd) * kMaxN + n];
-      }
+      v = seg == 0 ? (p.h0 ? p.h0[bd * N + n] : 0.f)
+                   : p.carry_h[((seg - 1) * p.batch * p.dim + bd) * kMaxN + n];
     }
-    h[k] = hin;
+    hin[k] = v;
   }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  const float dt_clamp = kMaxDecayArg / fmaxf(amax, 1e-30f);  // per channel
+  const float2 A01 = make_float2(A2[0], A2[1]);
+  const float2 A23 = make_float2(A2[2], A2[3]);
+  float2 h01 = make_float2(hin[0], hin[1]);
+  float2 h23 = make_float2(hin[2], hin[3]);
   const float biasd = (ch_ok && p.bias) ? p.bias[d] : 0.f;
   const float Dd = (ch_ok && p.D) ? p.D[d] : 0.f;
   float dtsum = 0.f;
+  const T* zrow = kGate && ch_ok ? static_cast<const T*>(p.z) + b * p.z_sb + d * p.z_sd : nullptr;
+  T* yrow = MODE == kFull && ch_ok ? static_cast<T*>(p.y) + b * p.y_sb + d * p.y_sd : nullptr;
 
   // ---- tile loads ----------------------------------------------------------------
   // Row r of a tile: [0, kCH) u, [kCH, 2kCH) delta, [2kCH, 2kCH + 16) B, then
-  // (full pass) 16 rows of C and, with a gate, kCH rows of z.
-  constexpr int kRowsAgg = 2 * kCH + kMaxN;
-  constexpr int kRows = MODE == kFull ? kRowsAgg + kMaxN + (HAS_Z ? kCH : 0) : kRowsAgg;
-  auto row_src = [&](int r, int buf, const T*& src, T*& dst) {
+  // (full pass) 16 rows of C.
+  constexpr int kRows = 2 * kCH + kMaxN + (MODE == kFull ? kMaxN : 0);
+  auto row_src = [&](int r, int ubuf, const T*& src, T*& dst) {
     if (r < kCH) {
       const int64_t dd = d0 + r;
       src = dd < p.dim ? gu + b * p.u_sb + dd * p.u_sd : nullptr;
-      dst = sm.raw_u[buf][r];
+      dst = sm.raw_u[ubuf][r];
     } else if (r < 2 * kCH) {
       const int64_t dd = d0 + r - kCH;
       src = dd < p.dim ? gdl + b * p.dl_sb + dd * p.dl_sd : nullptr;
-      dst = sm.raw_dl[buf][r - kCH];
+      dst = sm.raw_dl[r - kCH];
     } else if (r < 2 * kCH + kMaxN) {
       const int n = r - 2 * kCH;
       src = n < N ? gB + b * p.B_sb + n * p.B_sn : nullptr;
-      dst = sm.raw_B[buf][n];
-    } else if (r < 2 * kCH + 2 * kMaxN) {
+      dst = sm.raw_B[n];
+    } else {
       const int n = r - 2 * kCH - kMaxN;
       src = n < N ? gC + b * p.C_sb + n * p.C_sn : nullptr;
-      dst = sm.raw_C[buf][n];
-    } else {
-      const int64_t dd = d0 + r - 2 * kCH - 2 * kMaxN;
-      src = dd < p.dim ? gz + b * p.z_sb + dd * p.z_sd : nullptr;
-      dst = sm.raw_z[buf][r - 2 * kCH - 2 * kMaxN];
+      dst = sm.raw_C[n];
     }
   };
-  auto issue_load = [&](int buf, int64_t t0) {
+  auto issue_load = [&](int ubuf, int64_t t0) {
     const int len = static_cast<int>(imin64(kTL, l1 - t0));
     if (VEC) {
       for (int i = tid; i < kRows * kCPR; i += kThreads) {
@@ -167,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
         const int e = (i % kCPR) * kEPC;
         const T* src;
         T* dst;
-        row_src(r, buf, src, dst);
+        row_src(r, ubuf, src, dst);
         int nbytes = 0;
         const T* from = gu;  // any valid address when nothing is read
         if (src != nullptr && e < len) {
@@ -183,173 +305,196 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
         const int e = i % kTL;
         const T* src;
         T* dst;
-        row_src(r, buf, src, dst);
+        row_src(r, ubuf, src, dst);
         dst[e] = (src != nullptr && e < len) ? src[t0 + e] : from_f32<T>(0.f);
+      }
+    }
+  };
+
+  // z of the lane's epilogue steps of the tile starting at tt0, kept packed.
+  RawPair<T> zn[kGate ? kTL / kSub : 1];
+  auto prefetch_z = [&](RawPair<T>* dst, int64_t tt0) {
+    const int len = static_cast<int>(imin64(kTL, l1 - tt0));
+#pragma unroll
+    for (int s = 0; s < kTL / kSub; ++s) {
+      const int te = s * kSub + 2 * g;
+      dst[s] = RawPair<T>();
+      if (zrow != nullptr && te < len) {
+        if (VEC && te + 1 < len) {
+          dst[s].load(zrow + tt0 + te);
+        } else {
+          dst[s].load_scalar(zrow + tt0 + te, true, te + 1 < len);
+        }
       }
     }
   };
 
   const int64_t ntiles = l1 > l0 ? (l1 - l0 + kTL - 1) / kTL : 0;
   if (ntiles > 0) issue_load(0, l0);
+  if (kGate && ntiles > 0) prefetch_z(zn, l0);
 
   for (int64_t k = 0; k < ntiles; ++k) {
-    const int buf = static_cast<int>(k & 1);
+    const int ubuf = static_cast<int>(k & 1);
     const int64_t t0 = l0 + k * kTL;
     const int len = static_cast<int>(imin64(kTL, l1 - t0));
     if (VEC) cp_async_wait_all();
-    __syncthreads();  // tile k visible; the previous y tile has been stored
+    __syncthreads();  // tile k visible; every thread is done with tile k - 1
 
     // ---- per-tile preparation ------------------------------------------------------
-    {  // B (and C) to fp32, transposed to [t][n]
-      const int t = tid % kTL;
-      const int half = tid / kTL;  // states [8 half, 8 half + 8)
-      const int sw = bc_swizzle(t);
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int chunk = 2 * half + j;
-        float4 vb;
-        vb.x = to_f32(sm.raw_B[buf][4 * chunk + 0][t]);
-        vb.y = to_f32(sm.raw_B[buf][4 * chunk + 1][t]);
-        vb.z = to_f32(sm.raw_B[buf][4 * chunk + 2][t]);
-        vb.w = to_f32(sm.raw_B[buf][4 * chunk + 3][t]);
-        *reinterpret_cast<float4*>(&sm.Bf[t][4 * (chunk ^ sw)]) = vb;
-        if (MODE == kFull) {
-          float4 vc;
-          vc.x = to_f32(sm.raw_C[buf][4 * chunk + 0][t]);
-          vc.y = to_f32(sm.raw_C[buf][4 * chunk + 1][t]);
-          vc.z = to_f32(sm.raw_C[buf][4 * chunk + 2][t]);
-          vc.w = to_f32(sm.raw_C[buf][4 * chunk + 3][t]);
-          *reinterpret_cast<float4*>(&sm.Cf[t][4 * (chunk ^ sw)]) = vc;
-        }
+    {  // B and C to fp32, [step][state]: thread -> states 4q..4q+3, steps 2r, 2r+1
+      const int q = tid % 4;
+      const int r = tid / 4;
+      const float2 vb0 = load_pair<T>(&sm.raw_B[4 * q + 0][2 * r]);
+      const float2 vb1 = load_pair<T>(&sm.raw_B[4 * q + 1][2 * r]);
+      const float2 vb2 = load_pair<T>(&sm.raw_B[4 * q + 2][2 * r]);
+      const float2 vb3 = load_pair<T>(&sm.raw_B[4 * q + 3][2 * r]);
+      *reinterpret_cast<float4*>(&sm.Bf[2 * r][4 * q]) = make_float4(vb0.x, vb1.x, vb2.x, vb3.x);
+      *reinterpret_cast<float4*>(&sm.Bf[2 * r + 1][4 * q]) = make_float4(vb0.y, vb1.y, vb2.y, vb3.y);
+      if (MODE == kFull) {
+        const float2 vc0 = load_pair<T>(&sm.raw_C[4 * q + 0][2 * r]);
+        const float2 vc1 = load_pair<T>(&sm.raw_C[4 * q + 1][2 * r]);
+        const float2 vc2 = load_pair<T>(&sm.raw_C[4 * q + 2][2 * r]);
+        const float2 vc3 = load_pair<T>(&sm.raw_C[4 * q + 3][2 * r]);
+        *reinterpret_cast<float4*>(&sm.Cf[2 * r][4 * q]) = make_float4(vc0.x, vc1.x, vc2.x, vc3.x);
+        *reinterpret_cast<float4*>(&sm.Cf[2 * r + 1][4 * q]) =
+            make_float4(vc0.y, vc1.y, vc2.y, vc3.y);
       }
     }
     {  // dt' and dt' u for steps [16 g, 16 g + 16) of this thread's channel
       const int tq = g * (kTL / kNG);
 #pragma unroll
       for (int j = 0; j < kTL / kNG; j += 4) {
-        float4 vdt, vdu;
-        float* pdt = &vdt.x;
-        float* pdu = &vdu.x;
+        float vdt[4], vdu[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int t = tq + j + q;
-          const float s = to_f32(sm.raw_dl[buf][cl][t]) + biasd;
-          float dt = p.softplus ? softplus_f(s) : s;
-          dt = t < len ? dt : 0.f;  // steps past the end leave the state alone
-          pdt[q] = dt;
-          pdu[q] = dt * to_f32(sm.raw_u[buf][cl][t]);
+        for (int q2 = 0; q2 < 4; q2 += 2) {
+          const int t = tq + j + q2;
+          const float2 dl = load_pair<T>(&sm.raw_dl[cl][t]);
+          const float2 uv = load_pair<T>(&sm.raw_u[ubuf][cl][t]);
+          float2 s = __fadd2_rn(dl, make_float2(biasd, biasd));
+          if (p.softplus) s = softplus2(s);
+          s.x = t < len ? s.x : 0.f;  // steps past the end leave the state alone
+          s.y = t + 1 < len ? s.y : 0.f;
+          const float2 dv = __fmul2_rn(s, uv);
+          vdt[q2] = fminf(fmaxf(s.x, -dt_clamp), dt_clamp);
+          vdt[q2 + 1] = fminf(fmaxf(s.y, -dt_clamp), dt_clamp);
+          vdu[q2] = dv.x;
+          vdu[q2 + 1] = dv.y;
         }
-        *reinterpret_cast<float4*>(&sm.dtp[cl][tq + j]) = vdt;
-        *reinterpret_cast<float4*>(&sm.du[cl][tq + j]) = vdu;
+        *reinterpret_cast<float4*>(&sm.dtp[cl][tq + j]) = make_float4(vdt[0], vdt[1], vdt[2], vdt[3]);
+        *reinterpret_cast<float4*>(&sm.du[cl][tq + j]) = make_float4(vdu[0], vdu[1], vdu[2], vdu[3]);
       }
     }
     __syncthreads();
-    if (k + 1 < ntiles) issue_load(buf ^ 1, t0 + kTL);
+    if (k + 1 < ntiles) issue_load(ubuf ^ 1, t0 + kTL);
 
     // ---- the scan over this tile ---------------------------------------------------
-    const int nsub = (len + kSub - 1) / kSub;
-    for (int s = 0; s < nsub; ++s) {
+    // z for the lane's epilogue steps (8 s + 2 g + {0, 1}) of this tile was
+    // fetched during the previous tile; fetch the next tile's now.
+    RawPair<T> zt[kTL / kSub];
+    if (kGate) {
+#pragma unroll
+      for (int s = 0; s < kTL / kSub; ++s) zt[s] = zn[s];
+      if (k + 1 < ntiles) prefetch_z(zn, t0 + kTL);
+    }
+    const float* bf = &sm.Bf[0][kNPT * g];
+    const float* cf = &sm.Cf[0][kNPT * g];
+    // Every sub-tile of the tile is processed (steps past `len` carry dt' = 0 and
+    // dt' u = 0, which leave the state unchanged), so the loop unrolls fully.
+    // The decays of sub-tile s + 1 are computed while sub-tile s runs its
+    // recurrence and epilogue, which keeps the special-function pipe busy.
+    SubDecays dcur, dnext;
+    sub_decays(&sm.dtp[cl][0], A01, A23, dcur);
+#pragma unroll
+    for (int s = 0; s < kTL / kSub; ++s) {
       const int tb = s * kSub;
-      float dtv[kSub], duv[kSub];
-      *reinterpret_cast<float4*>(&dtv[0]) = *reinterpret_cast<const float4*>(&sm.dtp[cl][tb]);
-      *reinterpret_cast<float4*>(&dtv[4]) = *reinterpret_cast<const float4*>(&sm.dtp[cl][tb + 4]);
-      *reinterpret_cast<float4*>(&duv[0]) = *reinterpret_cast<const float4*>(&sm.du[cl][tb]);
-      *reinterpret_cast<float4*>(&duv[4]) = *reinterpret_cast<const float4*>(&sm.du[cl][tb + 4]);
-      float yp[kSub];
+      const int te = tb + 2 * g;  // this lane's two epilogue steps: te, te + 1
+      if (s + 1 < kTL / kSub) sub_decays(&sm.dtp[cl][tb + kSub], A01, A23, dnext);
+      float dus[kSub];
+      *reinterpret_cast<float4*>(&dus[0]) = *reinterpret_cast<const float4*>(&sm.du[cl][tb]);
+      *reinterpret_cast<float4*>(&dus[4]) = *reinterpret_cast<const float4*>(&sm.du[cl][tb + 4]);
+
+      // the recurrence
+      float ys[kSub];
 #pragma unroll
       for (int tt = 0; tt < kSub; ++tt) {
         const int t = tb + tt;
-        const int col = 4 * (g ^ bc_swizzle(t));
-        const float4 bq = *reinterpret_cast<const float4*>(&sm.Bf[t][col]);
-        const float bv[4] = {bq.x, bq.y, bq.z, bq.w};
+        const float4 bq = *reinterpret_cast<const float4*>(bf + t * kMaxN);
+        const float2 du2 = make_float2(dus[tt], dus[tt]);
+        h01 = __ffma2_rn(dcur.a01[tt], h01, __fmul2_rn(du2, make_float2(bq.x, bq.y)));
+        h23 = __ffma2_rn(dcur.a23[tt], h23, __fmul2_rn(du2, make_float2(bq.z, bq.w)));
         if (MODE == kFull) {
-          const float4 cq = *reinterpret_cast<const float4*>(&sm.Cf[t][col]);
-          const float cv[4] = {cq.x, cq.y, cq.z, cq.w};
-          float acc = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < kNPT; ++kk) {
-            const float dA = ex2_approx(dtv[tt] * A2[kk]);
-            h[kk] = fmaf(dA, h[kk], duv[tt] * bv[kk]);
-            acc = fmaf(cv[kk], h[kk], acc);
-          }
-          yp[tt] = acc;
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < kNPT; ++kk) {
-            const float dA = ex2_approx(dtv[tt] * A2[kk]);
-            h[kk] = fmaf(dA, h[kk], duv[tt] * bv[kk]);
-          }
-          dtsum += dtv[tt];
+          const float4 cq = *reinterpret_cast<const float4*>(cf + t * kMaxN);
+          float2 yv = __fmul2_rn(make_float2(cq.x, cq.y), h01);
+          yv = __ffma2_rn(make_float2(cq.z, cq.w), h23, yv);
+          ys[tt] = yv.x + yv.y;
         }
       }
-      if (MODE == kFull) {
-        *reinterpret_cast<float4*>(&sm.red[cl][g][0]) = make_float4(yp[0], yp[1], yp[2], yp[3]);
-        *reinterpret_cast<float4*>(&sm.red[cl][g][4]) = make_float4(yp[4], yp[5], yp[6], yp[7]);
-        __syncwarp();
-        float y0 = 0.f, y1 = 0.f;
+      if (MODE == kAgg) {
+        float dts[kSub];
+        *reinterpret_cast<float4*>(&dts[0]) = *reinterpret_cast<const float4*>(&sm.dtp[cl][tb]);
+        *reinterpret_cast<float4*>(&dts[4]) = *reinterpret_cast<const float4*>(&sm.dtp[cl][tb + 4]);
 #pragma unroll
-        for (int gg = 0; gg < kNG; ++gg) {
-          const float2 v = *reinterpret_cast<const float2*>(&sm.red[cl][gg][2 * g]);
-          y0 += v.x;
-          y1 += v.y;
-        }
-        __syncwarp();
-        const float ys[2] = {y0, y1};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int t = tb + 2 * g + i;
-          if (t < len) {
-            const float uv = to_f32(sm.raw_u[buf][cl][t]);
-            float yv = fmaf(Dd, uv, ys[i]);
-            if (kGate) yv *= silu_f(to_f32(sm.raw_z[buf][cl][t]));
-            sm.yout[cl][t] = from_f32<T>(yv);
-          }
-        }
+        for (int tt = 0; tt < kSub; ++tt) dtsum += dts[tt];
       }
-    }
 
-    // ---- store the y tile ------------------------------------------------------------
-    if (MODE == kFull) {
-      __syncthreads();
-      T* gy = static_cast<T*>(p.y);
-      if (VEC) {
-        for (int i = tid; i < kCH * kCPR; i += kThreads) {
-          const int r = i / kCPR;
-          const int e = (i % kCPR) * kEPC;
-          const int64_t dd = d0 + r;
-          if (dd >= p.dim || e >= len) continue;
-          T* dst = gy + b * p.y_sb + dd * p.y_sd + t0 + e;
-          if (e + kEPC <= len) {
-            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&sm.yout[r][e]);
+      if (MODE == kFull) {
+        // Reduce-scatter of the 8 partial sums over the channel's 4 lanes
+        // (butterfly over lane bits 1 then 0): lane g ends with the full sums
+        // of steps te = tb + 2 g and te + 1.
+        const bool hi2 = (g & 2) != 0;
+        float w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float send = hi2 ? ys[i] : ys[i + 4];
+          const float keep = hi2 ? ys[i + 4] : ys[i];
+          w[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        }
+        const bool hi1 = (g & 1) != 0;
+        float2 acc;
+        {
+          const float s0 = hi1 ? w[0] : w[2];
+          const float s1 = hi1 ? w[1] : w[3];
+          const float k0 = hi1 ? w[2] : w[0];
+          const float k1 = hi1 ? w[3] : w[1];
+          acc.x = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);
+          acc.y = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
+        }
+        if (yrow != nullptr && te < len) {
+          const float2 uv = load_pair<T>(&sm.raw_u[ubuf][cl][te]);
+          float y0 = fmaf(Dd, uv.x, acc.x);
+          float y1 = fmaf(Dd, uv.y, acc.y);
+          if (kGate) {
+            const float2 zv = zt[s].get();
+            y0 *= gate_silu<T>(zv.x);
+            y1 *= gate_silu<T>(zv.y);
+          }
+          if (VEC && te + 1 < len) {
+            store_pair<T>(yrow + t0 + te, y0, y1);
           } else {
-            for (int q = 0; q < len - e; ++q) dst[q] = sm.yout[r][e + q];
+            yrow[t0 + te] = from_f32<T>(y0);
+            if (te + 1 < len) yrow[t0 + te + 1] = from_f32<T>(y1);
           }
         }
-      } else {
-        for (int i = tid; i < kCH * kTL; i += kThreads) {
-          const int r = i / kTL;
-          const int e = i % kTL;
-          const int64_t dd = d0 + r;
-          if (dd < p.dim && e < len) gy[b * p.y_sb + dd * p.y_sd + t0 + e] = sm.yout[r][e];
-        }
       }
+      if (s + 1 < kTL / kSub) dcur = dnext;
     }
   }
 
   // ---- outgoing state ----------------------------------------------------------------
   if (!ch_ok) return;
+  const float hs[kNPT] = {h01.x, h01.y, h23.x, h23.y};
   if (MODE == kFull) {
     if (p.h_last != nullptr && seg == p.nseg - 1) {
 #pragma unroll
-      for (int k = 0; k < kNPT; ++k) {
-        const int n = g * kNPT + k;
-        if (n < N) p.h_last[bd * N + n] = h[k];
+      for (int kk = 0; kk < kNPT; ++kk) {
+        const int n = g * kNPT + kk;
+        if (n < N) p.h_last[bd * N + n] = hs[kk];
       }
     }
   } else {
     const int64_t slot = seg * p.batch * p.dim + bd;
 #pragma unroll
-    for (int k = 0; k < kNPT; ++k) p.carry_h[slot * kMaxN + g * kNPT + k] = h[k];
+    for (int kk = 0; kk < kNPT; ++kk) p.carry_h[slot * kMaxN + g * kNPT + kk] = hs[kk];
     if (g == 0) p.carry_dt[slot] = dtsum;
   }
 }
