@@ -18,7 +18,8 @@ bound by its exponentials and fp32 lane operations, not by HBM), the same
 metric end to end through the C ABI from pinned host buffers, clocks sampled
 during the timed region, the CPU oracle as a baseline, and (without --quick)
 one line per other workload: tiny fp32, the 2.8B-layer shape with and
-without gate, the 2^20-step sequence and the decode step.
+without gate, the 2^20-step sequence, the Mamba-2 chunked scan and the
+decode step.
 
 ``--impl reference`` times the CPU oracle instead, on a bounded sample of the
 same workload per step, with the same metric and unit.
@@ -46,6 +47,14 @@ MUFU_LANES_PER_SM = 16       # measured: 16.0 ex2 / lg2 / tanh per SM per clk
 EXP_POLY_LANE_OPS = 8        # FMA-pipe cost of one range-reduced degree-5 exp2
 
 
+def bf16_peak_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return 1590.0
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -67,6 +76,27 @@ def scan_bytes(batch, dim, dstate, seqlen, esize, gate=True, h_last=True):
     if h_last:
         total += batch * dim * dstate * 4
     return total
+
+
+def ssd_bytes(batch, seqlen, nheads, headdim, dstate, gate=False, h0=False):
+    """Algorithmic HBM bytes of one chunked scan (bf16 tensors, fp32 state)."""
+    x = batch * seqlen * nheads * headdim * 2
+    total = 2 * x + (x if gate else 0)               # x, y (, z)
+    total += 2 * batch * seqlen * dstate * 2          # B, C
+    total += batch * seqlen * nheads * 2              # delta
+    total += batch * nheads * headdim * dstate * 4 * (2 if h0 else 1)  # h_last (, h0)
+    total += 3 * nheads * 4
+    return total
+
+
+def ssd_flops(batch, seqlen, nheads, headdim, dstate, chunk):
+    """Dense tensor-core FLOPs of the chunked form: C B^T per (batch, chunk),
+    and per head the masked Q x Q product with X', the chunk state and the
+    read-out of the carried state."""
+    nc = -(-seqlen // chunk)
+    g = 2 * chunk * chunk * dstate
+    per_head = 2 * chunk * chunk * headdim + 2 * 2 * chunk * dstate * headdim
+    return batch * nc * (g + nheads * per_head)
 
 
 def alu_cycles_per_elem(dstate, gate=True, softplus=True):
@@ -348,6 +378,37 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
                     "launches_per_call": case.launches}
         del case
         torch.cuda.empty_cache()
+    # Mamba-2 chunked scan (tensor cores)
+    cfg = workload_cfg("mamba2_ssd")
+    sin = synth.make_ssd_inputs(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"],
+                                cfg["dstate"], cfg["dtype"], cfg["gate"], cfg["seed"], cfg["s_range"])
+    bfd = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)
+    f32d = lambda a: torch.from_numpy(a).cuda()
+    sx, sdl, sB, sC = bfd(sin["x"]), bfd(sin["delta"]), bfd(sin["B"]), bfd(sin["C"])
+    sA, sD, sbias = f32d(sin["A"]), f32d(sin["D"]), f32d(sin["delta_bias"])
+    sy = torch.empty_like(sx)
+    sh = torch.empty((cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"]),
+                     dtype=torch.float32, device="cuda")
+    sws = torch.empty(api.ssd_workspace_size(cfg["batch"], cfg["seqlen"], cfg["nheads"],
+                                             cfg["headdim"], cfg["dstate"], cfg["chunk"]),
+                      dtype=torch.uint8, device="cuda")
+    sstep = lambda: api.ssd_fwd(sx, sdl, sA, sB, sC, sD, None, sbias, True, None,
+                                chunk=cfg["chunk"], y=sy, h_last=sh, workspace=sws)
+    total, per, _ = time_steps(sstep, steps, warmup, flush, 1, None)
+    sec = total / steps
+    sb = ssd_bytes(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"])
+    sf = ssd_flops(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"],
+                   cfg["chunk"])
+    out["mamba2_ssd"] = {
+        "config": (f"batch={cfg['batch']} seqlen={cfg['seqlen']} nheads={cfg['nheads']} "
+                   f"headdim={cfg['headdim']} dstate={cfg['dstate']} chunk={cfg['chunk']} bf16"),
+        "us_per_call": round(sec * 1e6, 2), "GB_per_s": round(sb / sec / 1e9, 1),
+        "hbm_frac": round(sb / sec / 1e9 / hbm_peak, 4),
+        "TFLOP_per_s": round(sf / sec / 1e12, 1),
+        "tensor_frac_of_measured_bf16": round(sf / sec / 1e12 / bf16_peak_tflops(), 4),
+        "launches_per_call": 2}
+    del sx, sdl, sB, sC, sy, sws
+    torch.cuda.empty_cache()
     # decode step on the 2.8B-layer channel count (batch 4 x 5120 channels)
     cfg = workload_cfg("mamba2p8b_layer")
     B_, D_, N_ = cfg["batch"], cfg["dim"], cfg["dstate"]

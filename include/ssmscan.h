@@ -188,7 +188,18 @@ ssm_status_t ssm_scan_step(const ssm_step_args_t* args, ssm_stream_t stream);
  *   B, C        : (batch, seqlen, dstate)            `dtype` (shared by all heads)
  *   A, D, delta_bias : (nheads) fp32 (D, delta_bias may be NULL)
  *   h0, h_last  : (batch, nheads, headdim, dstate) fp32 or NULL.
- * chunk is the length of the intra-chunk quadratic block. */
+ * chunk is the length of the intra-chunk quadratic block; the result does
+ * not depend on it beyond rounding.
+ * Implemented: dtype SSM_BF16, dstate 128, headdim 64, chunk 128 or 256
+ * (others return SSM_ERR_UNSUPPORTED); x, B, C, z and y 16-byte aligned.
+ * The intra-chunk contractions run on the tensor cores with bf16 operands
+ * and fp32 accumulation; the state carried between chunks enters them in
+ * bf16 and is accumulated in fp32.
+ * Workspace (ssm_scan_fwd_chunked_workspace_size bytes, 256-byte aligned):
+ * its first int is a status word, zeroed by the call and set non-zero by the
+ * GPU if a bounded wait for a tensor-core result gave up (the outputs are
+ * then invalid); read it after the stream has finished.  The rest holds the
+ * state entering every chunk.  Calls sharing a workspace must not overlap. */
 typedef struct {
   int64_t batch, seqlen, nheads, headdim, dstate, chunk;
   ssm_dtype_t dtype;

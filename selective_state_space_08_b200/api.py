@@ -166,3 +166,69 @@ def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_s
     a.state, a.y = _ptr(state), _ptr(y)
     _abi.check(_abi.load().ssm_scan_step(ctypes.byref(a), _stream(stream)), "ssm_scan_step")
     return y
+
+
+def ssd_workspace_size(batch, seqlen, nheads, headdim, dstate, chunk) -> int:
+    a = _abi.SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.chunk = (batch, seqlen, nheads, headdim,
+                                                                  dstate, chunk)
+    a.dtype = _abi.SSM_BF16
+    n = _abi.load().ssm_scan_fwd_chunked_workspace_size(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported or invalid sizes")
+    return int(n)
+
+
+def ssd_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True, h0=None, *,
+            chunk=256, y=None, h_last=None, return_last_state=True, workspace=None, stream=None,
+            check_status=False):
+    """Mamba-2 scalar-decay scan, chunked (tensor cores).
+
+    x, z: (batch, L, H, P) bfloat16; delta: (batch, L, H) bfloat16; B, C:
+    (batch, L, N) bfloat16; A, D, delta_bias: (H,) float32; h0: (batch, H, P, N)
+    float32.  Returns (y, h_last).  With ``check_status`` the call waits for the
+    GPU and raises if a tensor-core wait inside the kernels gave up."""
+    for name, t in (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+        _cuda(name, t)
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    batch, L, H, P = x.shape
+    N = B.shape[-1]
+    for name, t, shape, dtype in (("x", x, (batch, L, H, P), torch.bfloat16),
+                                  ("delta", delta, (batch, L, H), torch.bfloat16),
+                                  ("B", B, (batch, L, N), torch.bfloat16),
+                                  ("C", C, (batch, L, N), torch.bfloat16),
+                                  ("z", z, (batch, L, H, P), torch.bfloat16),
+                                  ("A", A, (H,), torch.float32), ("D", D, (H,), torch.float32),
+                                  ("delta_bias", delta_bias, (H,), torch.float32),
+                                  ("h0", h0, (batch, H, P, N), torch.float32),
+                                  ("h_last", h_last, (batch, H, P, N), torch.float32)):
+        if t is not None and (tuple(t.shape) != shape or t.dtype != dtype):
+            raise ValueError(f"{name} must be {dtype} of shape {shape}")
+    if y is None:
+        y = torch.empty_like(x)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((batch, H, P, N), dtype=torch.float32, device=x.device)
+    a = _abi.SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.chunk = batch, L, H, P, N, chunk
+    a.dtype = _abi.SSM_BF16
+    a.x, a.delta, a.A, a.B, a.C, a.D = _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D)
+    a.delta_bias, a.delta_softplus, a.z = _ptr(delta_bias), 1 if delta_softplus else 0, _ptr(z)
+    a.h0, a.y, a.h_last = _ptr(h0), _ptr(y), _ptr(h_last)
+    lib = _abi.load()
+    need = lib.ssm_scan_fwd_chunked_workspace_size(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise ValueError("unsupported or invalid arguments")
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(int(need), dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _abi.check(lib.ssm_scan_fwd_chunked(ctypes.byref(a), _ptr(workspace), ws_bytes,
+                                        _stream(stream)), "ssm_scan_fwd_chunked")
+    if check_status:
+        torch.cuda.synchronize(x.device)
+        status = int(workspace[:4].view(torch.int32).item())
+        if status != 0:
+            raise RuntimeError(f"ssm_scan_fwd_chunked: device status {status} "
+                               "(a tensor-core wait gave up)")
+    return y, h_last

@@ -12,6 +12,7 @@
 #include "../../include/ssmscan.h"
 #include "scan_fwd.cuh"
 #include "scan_step.cuh"
+#include "ssd_fwd.cuh"
 
 namespace {
 
@@ -220,6 +221,86 @@ ssm_status_t run_step(const StepParams& p, bool vec4, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------------------
+// Mamba-2 chunked scan
+// ---------------------------------------------------------------------------
+constexpr size_t kSsdStatusBytes = 256;  // status word at the start of the workspace
+
+ssm_status_t plan_ssd(const ssm_ssd_args_t* a, SsdParams* p, size_t* ws_bytes, bool check_ptrs) {
+  if (a == nullptr) return SSM_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->seqlen < 0 || a->nheads < 0 || a->headdim < 0 || a->dstate < 0)
+    return SSM_ERR_INVALID_ARG;
+  if (a->dtype != SSM_F32 && a->dtype != SSM_BF16) return SSM_ERR_INVALID_ARG;
+  if (a->dtype != SSM_BF16) return SSM_ERR_UNSUPPORTED;
+  if (a->dstate != ssd::kN || a->headdim != ssd::kP) return SSM_ERR_UNSUPPORTED;
+  if (a->chunk != 128 && a->chunk != 256) return SSM_ERR_UNSUPPORTED;
+  if (a->batch > 65535 || a->nheads > 65535) return SSM_ERR_UNSUPPORTED;
+  const bool any = a->batch > 0 && a->nheads > 0;
+  if (any && check_ptrs) {
+    if (a->A == nullptr) return SSM_ERR_INVALID_ARG;
+    if (a->seqlen > 0 && (a->x == nullptr || a->delta == nullptr || a->B == nullptr ||
+                          a->C == nullptr || a->y == nullptr))
+      return SSM_ERR_INVALID_ARG;
+  }
+  const void* vec[] = {a->x, a->B, a->C, a->y, a->z};
+  for (const void* t : vec)
+    if (t != nullptr && !aligned(t, 16)) return SSM_ERR_ALIGNMENT;
+  if (a->delta != nullptr && !aligned(a->delta, 2)) return SSM_ERR_ALIGNMENT;
+  const void* f32s[] = {a->A, a->D, a->delta_bias, a->h0, a->h_last};
+  for (const void* t : f32s)
+    if (t != nullptr && !aligned(t, 4)) return SSM_ERR_ALIGNMENT;
+  p->batch = a->batch;
+  p->seqlen = a->seqlen;
+  p->nheads = a->nheads;
+  p->headdim = a->headdim;
+  p->dstate = a->dstate;
+  p->chunk = a->chunk;
+  p->nchunks = (a->seqlen + a->chunk - 1) / a->chunk;
+  if (p->nchunks > 2147483647) return SSM_ERR_UNSUPPORTED;
+  p->x = static_cast<const __nv_bfloat16*>(a->x);
+  p->delta = static_cast<const __nv_bfloat16*>(a->delta);
+  p->A = a->A;
+  p->B = static_cast<const __nv_bfloat16*>(a->B);
+  p->C = static_cast<const __nv_bfloat16*>(a->C);
+  p->D = a->D;
+  p->bias = a->delta_bias;
+  p->softplus = a->delta_softplus ? 1 : 0;
+  p->z = static_cast<const __nv_bfloat16*>(a->z);
+  p->h0 = a->h0;
+  p->y = static_cast<__nv_bfloat16*>(a->y);
+  p->h_last = a->h_last;
+  *ws_bytes = kSsdStatusBytes + static_cast<size_t>(a->batch) * a->nheads * p->nchunks *
+                                    ssd::kN * ssd::kP * sizeof(__nv_bfloat16);
+  return SSM_OK;
+}
+
+template <int Q>
+ssm_status_t run_ssd(const SsdParams& p, cudaStream_t stream) {
+  auto state = ssd::ssd_state_kernel<Q>;
+  const size_t smem_state = sizeof(ssd::StateSmem<Q>) + 1024;
+  ssm_status_t st = cuda_status(set_smem(reinterpret_cast<const void*>(state), smem_state),
+                                "ssd: shared-memory opt-in");
+  if (st != SSM_OK) return st;
+  state<<<static_cast<unsigned>(p.batch * p.nheads), ssd::kThreads, smem_state, stream>>>(p);
+  st = cuda_status(cudaGetLastError(), "ssd: state pass launch");
+  if (st != SSM_OK || p.nchunks == 0) return st;
+  const size_t smem_scan = sizeof(ssd::ScanSmem<Q>) + 1024;
+  const dim3 grid(static_cast<unsigned>(p.nchunks), static_cast<unsigned>(p.nheads),
+                  static_cast<unsigned>(p.batch));
+  if (p.z != nullptr) {
+    auto scan = ssd::ssd_scan_kernel<Q, true>;
+    st = cuda_status(set_smem(reinterpret_cast<const void*>(scan), smem_scan), "ssd: opt-in");
+    if (st != SSM_OK) return st;
+    scan<<<grid, ssd::kThreads, smem_scan, stream>>>(p);
+  } else {
+    auto scan = ssd::ssd_scan_kernel<Q, false>;
+    st = cuda_status(set_smem(reinterpret_cast<const void*>(scan), smem_scan), "ssd: opt-in");
+    if (st != SSM_OK) return st;
+    scan<<<grid, ssd::kThreads, smem_scan, stream>>>(p);
+  }
+  return cuda_status(cudaGetLastError(), "ssd: chunk scan launch");
+}
+
+// ---------------------------------------------------------------------------
 // Static scratch for ssm_scan_fwd_noalloc.  In host code the name below is a
 // host-side stand-in, not a device address: the address kernels must use is
 // looked up with cudaGetSymbolAddress, once per device.
@@ -337,17 +418,27 @@ ssm_status_t ssm_scan_step(const ssm_step_args_t* a, ssm_stream_t stream_) {
 }
 
 size_t ssm_scan_fwd_chunked_workspace_size(const ssm_ssd_args_t* args) {
-  (void)args;
-  return static_cast<size_t>(-1);
+  SsdParams p;
+  size_t ws = 0;
+  if (plan_ssd(args, &p, &ws, false) != SSM_OK) return static_cast<size_t>(-1);
+  return ws;
 }
 
 ssm_status_t ssm_scan_fwd_chunked(const ssm_ssd_args_t* args, void* workspace,
-                                  size_t workspace_bytes, ssm_stream_t stream) {
-  (void)args;
-  (void)workspace;
-  (void)workspace_bytes;
-  (void)stream;
-  return SSM_ERR_UNSUPPORTED;
+                                  size_t workspace_bytes, ssm_stream_t stream_) {
+  SsdParams p;
+  size_t ws = 0;
+  ssm_status_t st = plan_ssd(args, &p, &ws, true);
+  if (st != SSM_OK) return st;
+  if (p.batch == 0 || p.nheads == 0) return SSM_OK;
+  if (workspace == nullptr || workspace_bytes < ws) return SSM_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return SSM_ERR_ALIGNMENT;
+  p.status = static_cast<int*>(workspace);
+  p.sprev = reinterpret_cast<__nv_bfloat16*>(static_cast<unsigned char*>(workspace) + kSsdStatusBytes);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  st = cuda_status(cudaMemsetAsync(p.status, 0, sizeof(int), stream), "ssd: status reset");
+  if (st != SSM_OK) return st;
+  return p.chunk == 256 ? run_ssd<256>(p, stream) : run_ssd<128>(p, stream);
 }
 
 const char* ssm_status_string(ssm_status_t s) {
