@@ -268,24 +268,50 @@ ssm_status_t plan_ssd(const ssm_ssd_args_t* a, SsdParams* p, size_t* ws_bytes, b
   p->h0 = a->h0;
   p->y = static_cast<__nv_bfloat16*>(a->y);
   p->h_last = a->h_last;
-  *ws_bytes = kSsdStatusBytes + static_cast<size_t>(a->batch) * a->nheads * p->nchunks *
-                                    ssd::kN * ssd::kP * sizeof(__nv_bfloat16);
+  const size_t states = static_cast<size_t>(a->batch) * a->nheads * p->nchunks * ssd::kN * ssd::kP;
+  const size_t cums = (static_cast<size_t>(a->batch) * a->nheads * p->nchunks * sizeof(float) + 255) /
+                      256 * 256;
+  *ws_bytes = kSsdStatusBytes + states * sizeof(float) + cums + states * sizeof(__nv_bfloat16);
+  // Heads per block: the chunk-state and scan kernels run one block per SM;
+  // choose the group that minimises (rounds of blocks) x (heads per block + the
+  // shared C B^T product, worth about 1.5 heads).
+  const int64_t sms = device_sm_count();
+  int64_t best = 1;
+  double best_cost = 1e300;
+  for (int64_t g = 1; g <= a->nheads && g <= ssd::kMaxGroup; ++g) {
+    const int64_t groups = (a->nheads + g - 1) / g;
+    if (g > 1 && (a->nheads + g - 2) / (g - 1) == groups) continue;  // same split, more heads
+    const int64_t blocks = a->batch * p->nchunks * groups;
+    const int64_t rounds = blocks == 0 ? 0 : (blocks + sms - 1) / sms;
+    const double cost = static_cast<double>(rounds) * (static_cast<double>(g) + 1.5);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = g;
+    }
+  }
+  p->hgroup = best;
   return SSM_OK;
 }
 
 template <int Q>
 ssm_status_t run_ssd(const SsdParams& p, cudaStream_t stream) {
-  auto state = ssd::ssd_state_kernel<Q>;
-  const size_t smem_state = sizeof(ssd::StateSmem<Q>) + 1024;
-  ssm_status_t st = cuda_status(set_smem(reinterpret_cast<const void*>(state), smem_state),
-                                "ssd: shared-memory opt-in");
-  if (st != SSM_OK) return st;
-  state<<<static_cast<unsigned>(p.batch * p.nheads), ssd::kThreads, smem_state, stream>>>(p);
+  ssm_status_t st = SSM_OK;
+  const unsigned groups = static_cast<unsigned>((p.nheads + p.hgroup - 1) / p.hgroup);
+  const dim3 grid(groups, static_cast<unsigned>(p.nchunks), static_cast<unsigned>(p.batch));
+  if (p.nchunks > 0) {
+    auto chunk_state = ssd::ssd_chunk_state_kernel<Q>;
+    const size_t smem = sizeof(ssd::ChunkStateSmem<Q>) + 1024;
+    st = cuda_status(set_smem(reinterpret_cast<const void*>(chunk_state), smem), "ssd: opt-in");
+    if (st != SSM_OK) return st;
+    chunk_state<<<grid, ssd::kThreads, smem, stream>>>(p);
+    st = cuda_status(cudaGetLastError(), "ssd: chunk-state launch");
+    if (st != SSM_OK) return st;
+  }
+  const int64_t elems = p.batch * p.nheads * ssd::kP * ssd::kN;
+  ssd::ssd_pass_kernel<<<static_cast<unsigned>((elems + 255) / 256), 256, 0, stream>>>(p);
   st = cuda_status(cudaGetLastError(), "ssd: state pass launch");
   if (st != SSM_OK || p.nchunks == 0) return st;
   const size_t smem_scan = sizeof(ssd::ScanSmem<Q>) + 1024;
-  const dim3 grid(static_cast<unsigned>(p.nchunks), static_cast<unsigned>(p.nheads),
-                  static_cast<unsigned>(p.batch));
   if (p.z != nullptr) {
     auto scan = ssd::ssd_scan_kernel<Q, true>;
     st = cuda_status(set_smem(reinterpret_cast<const void*>(scan), smem_scan), "ssd: opt-in");
@@ -433,8 +459,14 @@ ssm_status_t ssm_scan_fwd_chunked(const ssm_ssd_args_t* args, void* workspace,
   if (p.batch == 0 || p.nheads == 0) return SSM_OK;
   if (workspace == nullptr || workspace_bytes < ws) return SSM_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return SSM_ERR_ALIGNMENT;
-  p.status = static_cast<int*>(workspace);
-  p.sprev = reinterpret_cast<__nv_bfloat16*>(static_cast<unsigned char*>(workspace) + kSsdStatusBytes);
+  unsigned char* w = static_cast<unsigned char*>(workspace);
+  const size_t states = static_cast<size_t>(p.batch) * p.nheads * p.nchunks * ssd::kN * ssd::kP;
+  const size_t cums = (static_cast<size_t>(p.batch) * p.nheads * p.nchunks * sizeof(float) + 255) /
+                      256 * 256;
+  p.status = reinterpret_cast<int*>(w);
+  p.sloc = reinterpret_cast<float*>(w + kSsdStatusBytes);
+  p.cum_end = reinterpret_cast<float*>(w + kSsdStatusBytes + states * sizeof(float));
+  p.sprev = reinterpret_cast<__nv_bfloat16*>(w + kSsdStatusBytes + states * sizeof(float) + cums);
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   st = cuda_status(cudaMemsetAsync(p.status, 0, sizeof(int), stream), "ssd: status reset");
   if (st != SSM_OK) return st;
