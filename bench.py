@@ -47,6 +47,31 @@ MUFU_LANES_PER_SM = 16       # measured: 16.0 ex2 / lg2 / tanh per SM per clk
 EXP_POLY_LANE_OPS = 8        # FMA-pipe cost of one range-reduced degree-5 exp2
 
 
+SCAN_SOURCES = ["scan_fwd.cuh", "common.cuh", "exp2_poly.cuh"]
+
+
+def captured_traffic():
+    """DRAM bytes per launch of the scan kernel from the recorded ncu capture,
+    or None when the kernel sources changed since that capture."""
+    import hashlib
+    rec = {}
+    try:
+        with open(os.path.join(ROOT, "profiles", "scan_fwd_traffic.txt")) as f:
+            for line in f:
+                if line.strip() and not line.startswith("#"):
+                    k, v = line.split()
+                    rec[k] = v
+        h = hashlib.sha256()
+        for name in SCAN_SOURCES:
+            with open(os.path.join(ROOT, "selective_state_space_08_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+    except (OSError, ValueError):
+        return None
+    if rec.get("sources_sha256") != h.hexdigest():
+        return None
+    return int(rec["dram_bytes_per_launch"])
+
+
 def bf16_peak_tflops():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -465,7 +490,9 @@ def run_ours(args):
         "hbm_peak_gbs": hbm_peak, "hbm_peak_kind": peak_kind,
         "roofline": {"bound": "alu", "achieved": round(case.elems / kernel_s / 1e9, 2),
                      "peak": round(alu_peak / 1e9, 2), "unit": "Gelem/s",
-                     "frac": round(case.elems / kernel_s / alu_peak, 4), "traffic": None,
+                     "frac": round(case.elems / kernel_s / alu_peak, 4),
+                     "traffic": captured_traffic(),
+                     "traffic_unit": "bytes per launch (dram read + write, ncu)",
                      "kernel": "scan_fwd_kernel<bf16, full, gate>",
                      "hbm_achieved_gbs": round(case.bytes / kernel_s / 1e9, 1),
                      "hbm_frac": round(case.bytes / kernel_s / 1e9 / hbm_peak, 4),
