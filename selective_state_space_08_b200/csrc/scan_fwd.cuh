@@ -80,19 +80,25 @@ constexpr int kFull = 0, kAgg = 1;
 // |dt' A log2(e)| is clamped to this before the decay exponential: beyond it
 // the decay is below 2^-126 (or the state overflows anyway).
 constexpr float kMaxDecayArg = 126.0f;
+// fp32 B / C rows of 20 floats: the prep's stores of 8 consecutive steps from
+// one quarter-warp then land in 8 distinct 4-bank groups.
+constexpr int kBCRow = kMaxN + 4;
 
 template <typename T>
 struct Smem {
   static constexpr int kEPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
-  static constexpr int kRow = kTL + kEPC;            // raw row: tile + 16-byte pad
+  // A raw row holds a tile plus a 16-byte pad, so consecutive rows start 4
+  // banks apart: 8 lanes reading 16 bytes from 8 consecutive rows hit 32
+  // distinct banks.
+  static constexpr int kRow = kTL + kEPC;
   T raw_u[2][kCH][kRow];     // u is read again by the epilogue: two buffers
   T raw_dl[kCH][kRow];       // delta, B, C are consumed by the per-tile prep
   T raw_B[kMaxN][kRow];
   T raw_C[kMaxN][kRow];
   float dtp[kCH][kTL + 4];   // dt', clamped, per (channel, step): decay argument
   float du[kCH][kTL + 4];    // dt' * u
-  float Bf[kTL][kMaxN];      // fp32 B, [step][state]
-  float Cf[kTL][kMaxN];
+  float Bf[kTL][kBCRow];     // fp32 B, [step][state]
+  float Cf[kTL][kBCRow];
 };
 
 // softplus for a pair (see softplus_f in common.cuh for the three ranges; the
@@ -153,6 +159,63 @@ __device__ __forceinline__ void store_pair<float>(float* p, float a, float b) {
   *reinterpret_cast<float2*>(p) = make_float2(a, b);
 }
 
+// Eight consecutive elements of a shared-memory row (aligned to 8 elements) as fp32.
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(ws[i] << 16);
+    v[2 * i + 1] = __uint_as_float(ws[i] & 0xffff0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Stages rows [0, NROWS) x steps [t0, t0 + kTL) of a (row, time) array into
+// dst ([NROWS][kRow]); rows >= nvalid and steps >= len are zero-filled.
+// Thread tid copies the 16-byte chunk (tid % chunks-per-row) of rows
+// tid / chunks-per-row + k * rows-per-pass, so the row pattern is fixed at
+// compile time.
+template <typename T, int NROWS>
+__device__ __forceinline__ void copy_rows_async(T* dst, const T* base, int64_t rstride,
+                                                int nvalid, int64_t t0, int len,
+                                                const T* any_valid, int tid) {
+  constexpr int kEPC = Smem<T>::kEPC;
+  constexpr int kRow = Smem<T>::kRow;
+  constexpr int kCPR = kTL / kEPC;
+  constexpr int kRPP = kThreads / kCPR;
+  static_assert(NROWS % kRPP == 0, "rows per pass must divide the row count");
+  const int ce = (tid % kCPR) * kEPC;
+  const int r0 = tid / kCPR;
+  const int left = len - ce;
+  const int bytes = left <= 0 ? 0 : (left >= kEPC ? 16 : left * static_cast<int>(sizeof(T)));
+#pragma unroll
+  for (int k = 0; k < NROWS / kRPP; ++k) {
+    const int r = r0 + k * kRPP;
+    const bool ok = r < nvalid && bytes > 0;
+    cp_async16(dst + r * kRow + ce, ok ? base + r * rstride + t0 + ce : any_valid, ok ? bytes : 0);
+  }
+}
+template <typename T, int NROWS>
+__device__ __forceinline__ void copy_rows_scalar(T* dst, const T* base, int64_t rstride,
+                                                 int nvalid, int64_t t0, int len, int tid) {
+  constexpr int kRow = Smem<T>::kRow;
+  for (int i = tid; i < NROWS * kTL; i += kThreads) {
+    const int r = i / kTL;
+    const int e = i % kTL;
+    dst[r * kRow + e] = (r < nvalid && e < len) ? base[r * rstride + t0 + e] : from_f32<T>(0.f);
+  }
+}
+
 // Two consecutive elements kept in their storage format until used.
 template <typename T>
 struct RawPair;
@@ -207,8 +270,6 @@ template <typename T, int MODE, bool HAS_Z, bool VEC>
 __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem<T>& sm = *reinterpret_cast<Smem<T>*>(smem_raw);
-  constexpr int kEPC = Smem<T>::kEPC;
-  constexpr int kCPR = kTL / kEPC;  // 16-byte chunks per raw row
   constexpr bool kGate = HAS_Z && MODE == kFull;
 
   const int tid = threadIdx.x;
@@ -231,13 +292,11 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
 
   // ---- per-thread constants and incoming state -------------------------------
   float A2[kNPT], hin[kNPT];
-  float amax = 0.f;
 #pragma unroll
   for (int k = 0; k < kNPT; ++k) {
     const int n = g * kNPT + k;
     const bool ok = ch_ok && n < N;
     A2[k] = ok ? p.A[d * N + n] * kLog2e : 0.f;
-    amax = fmaxf(amax, fabsf(A2[k]));
     float v = 0.f;
     if (MODE == kFull && ok) {
       v = seg == 0 ? (p.h0 ? p.h0[bd * N + n] : 0.f)
@@ -245,69 +304,45 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
     }
     hin[k] = v;
   }
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  const float dt_clamp = kMaxDecayArg / fmaxf(amax, 1e-30f);  // per channel
   const float2 A01 = make_float2(A2[0], A2[1]);
   const float2 A23 = make_float2(A2[2], A2[3]);
   float2 h01 = make_float2(hin[0], hin[1]);
   float2 h23 = make_float2(hin[2], hin[3]);
-  const float biasd = (ch_ok && p.bias) ? p.bias[d] : 0.f;
   const float Dd = (ch_ok && p.D) ? p.D[d] : 0.f;
   float dtsum = 0.f;
   const T* zrow = kGate && ch_ok ? static_cast<const T*>(p.z) + b * p.z_sb + d * p.z_sd : nullptr;
   T* yrow = MODE == kFull && ch_ok ? static_cast<T*>(p.y) + b * p.y_sb + d * p.y_sd : nullptr;
 
+  // ---- per-thread constants of the dt' prep: channel pc, steps [pt0, pt0 + 16) ----
+  const int pc = tid % kCH;
+  const int pt0 = (tid / kCH) * (kTL / kNG);
+  float pbias = 0.f, pamax = 0.f;
+  if (d0 + pc < p.dim) {
+    const int64_t dp = d0 + pc;
+    pbias = p.bias ? p.bias[dp] : 0.f;
+    for (int n = 0; n < N; ++n) pamax = fmaxf(pamax, fabsf(p.A[dp * N + n] * kLog2e));
+  }
+  const float pclamp = kMaxDecayArg / fmaxf(pamax, 1e-30f);
+
   // ---- tile loads ----------------------------------------------------------------
-  // Row r of a tile: [0, kCH) u, [kCH, 2kCH) delta, [2kCH, 2kCH + 16) B, then
-  // (full pass) 16 rows of C.
-  constexpr int kRows = 2 * kCH + kMaxN + (MODE == kFull ? kMaxN : 0);
-  auto row_src = [&](int r, int ubuf, const T*& src, T*& dst) {
-    if (r < kCH) {
-      const int64_t dd = d0 + r;
-      src = dd < p.dim ? gu + b * p.u_sb + dd * p.u_sd : nullptr;
-      dst = sm.raw_u[ubuf][r];
-    } else if (r < 2 * kCH) {
-      const int64_t dd = d0 + r - kCH;
-      src = dd < p.dim ? gdl + b * p.dl_sb + dd * p.dl_sd : nullptr;
-      dst = sm.raw_dl[r - kCH];
-    } else if (r < 2 * kCH + kMaxN) {
-      const int n = r - 2 * kCH;
-      src = n < N ? gB + b * p.B_sb + n * p.B_sn : nullptr;
-      dst = sm.raw_B[n];
-    } else {
-      const int n = r - 2 * kCH - kMaxN;
-      src = n < N ? gC + b * p.C_sb + n * p.C_sn : nullptr;
-      dst = sm.raw_C[n];
-    }
-  };
+  const int nch = static_cast<int>(imin64(kCH, p.dim - d0));  // valid channels
+  const T* tu = gu + b * p.u_sb + d0 * p.u_sd;
+  const T* tdl = gdl + b * p.dl_sb + d0 * p.dl_sd;
+  const T* tB = gB + b * p.B_sb;
+  const T* tC = gC + b * p.C_sb;
   auto issue_load = [&](int ubuf, int64_t t0) {
     const int len = static_cast<int>(imin64(kTL, l1 - t0));
     if (VEC) {
-      for (int i = tid; i < kRows * kCPR; i += kThreads) {
-        const int r = i / kCPR;
-        const int e = (i % kCPR) * kEPC;
-        const T* src;
-        T* dst;
-        row_src(r, ubuf, src, dst);
-        int nbytes = 0;
-        const T* from = gu;  // any valid address when nothing is read
-        if (src != nullptr && e < len) {
-          nbytes = min(kEPC, len - e) * static_cast<int>(sizeof(T));
-          from = src + t0 + e;
-        }
-        cp_async16(dst + e, from, nbytes);
-      }
+      copy_rows_async<T, kCH>(&sm.raw_u[ubuf][0][0], tu, p.u_sd, nch, t0, len, gu, tid);
+      copy_rows_async<T, kCH>(&sm.raw_dl[0][0], tdl, p.dl_sd, nch, t0, len, gu, tid);
+      copy_rows_async<T, kMaxN>(&sm.raw_B[0][0], tB, p.B_sn, N, t0, len, gu, tid);
+      if (MODE == kFull) copy_rows_async<T, kMaxN>(&sm.raw_C[0][0], tC, p.C_sn, N, t0, len, gu, tid);
       cp_async_commit();
     } else {
-      for (int i = tid; i < kRows * kTL; i += kThreads) {
-        const int r = i / kTL;
-        const int e = i % kTL;
-        const T* src;
-        T* dst;
-        row_src(r, ubuf, src, dst);
-        dst[e] = (src != nullptr && e < len) ? src[t0 + e] : from_f32<T>(0.f);
-      }
+      copy_rows_scalar<T, kCH>(&sm.raw_u[ubuf][0][0], tu, p.u_sd, nch, t0, len, tid);
+      copy_rows_scalar<T, kCH>(&sm.raw_dl[0][0], tdl, p.dl_sd, nch, t0, len, tid);
+      copy_rows_scalar<T, kMaxN>(&sm.raw_B[0][0], tB, p.B_sn, N, t0, len, tid);
+      if (MODE == kFull) copy_rows_scalar<T, kMaxN>(&sm.raw_C[0][0], tC, p.C_sn, N, t0, len, tid);
     }
   };
 
@@ -341,47 +376,45 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
     __syncthreads();  // tile k visible; every thread is done with tile k - 1
 
     // ---- per-tile preparation ------------------------------------------------------
-    {  // B and C to fp32, [step][state]: thread -> states 4q..4q+3, steps 2r, 2r+1
-      const int q = tid % 4;
-      const int r = tid / 4;
-      const float2 vb0 = load_pair<T>(&sm.raw_B[4 * q + 0][2 * r]);
-      const float2 vb1 = load_pair<T>(&sm.raw_B[4 * q + 1][2 * r]);
-      const float2 vb2 = load_pair<T>(&sm.raw_B[4 * q + 2][2 * r]);
-      const float2 vb3 = load_pair<T>(&sm.raw_B[4 * q + 3][2 * r]);
-      *reinterpret_cast<float4*>(&sm.Bf[2 * r][4 * q]) = make_float4(vb0.x, vb1.x, vb2.x, vb3.x);
-      *reinterpret_cast<float4*>(&sm.Bf[2 * r + 1][4 * q]) = make_float4(vb0.y, vb1.y, vb2.y, vb3.y);
-      if (MODE == kFull) {
-        const float2 vc0 = load_pair<T>(&sm.raw_C[4 * q + 0][2 * r]);
-        const float2 vc1 = load_pair<T>(&sm.raw_C[4 * q + 1][2 * r]);
-        const float2 vc2 = load_pair<T>(&sm.raw_C[4 * q + 2][2 * r]);
-        const float2 vc3 = load_pair<T>(&sm.raw_C[4 * q + 3][2 * r]);
-        *reinterpret_cast<float4*>(&sm.Cf[2 * r][4 * q]) = make_float4(vc0.x, vc1.x, vc2.x, vc3.x);
-        *reinterpret_cast<float4*>(&sm.Cf[2 * r + 1][4 * q]) =
-            make_float4(vc0.y, vc1.y, vc2.y, vc3.y);
+    {  // B and C to fp32, [step][state]: thread -> states 4q .. 4q+3, steps r and r + 32
+      static_assert(kThreads == 128 && kTL == 64 && kMaxN == 16, "prep mapping");
+      const int r = tid % 32;
+      const int q = tid / 32;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = r + 32 * h;
+        *reinterpret_cast<float4*>(&sm.Bf[t][4 * q]) =
+            make_float4(to_f32<T>(sm.raw_B[4 * q + 0][t]), to_f32<T>(sm.raw_B[4 * q + 1][t]),
+                        to_f32<T>(sm.raw_B[4 * q + 2][t]), to_f32<T>(sm.raw_B[4 * q + 3][t]));
+        if (MODE == kFull)
+          *reinterpret_cast<float4*>(&sm.Cf[t][4 * q]) =
+              make_float4(to_f32<T>(sm.raw_C[4 * q + 0][t]), to_f32<T>(sm.raw_C[4 * q + 1][t]),
+                          to_f32<T>(sm.raw_C[4 * q + 2][t]), to_f32<T>(sm.raw_C[4 * q + 3][t]));
       }
     }
-    {  // dt' and dt' u for steps [16 g, 16 g + 16) of this thread's channel
-      const int tq = g * (kTL / kNG);
+    {  // dt' and dt' u of channel pc, steps [pt0, pt0 + 16)
 #pragma unroll
-      for (int j = 0; j < kTL / kNG; j += 4) {
-        float vdt[4], vdu[4];
+      for (int jj = 0; jj < kTL / kNG; jj += 8) {
+        const int t = pt0 + jj;
+        float dl[8], uv[8], vdt[8], vdu[8];
+        load8<T>(&sm.raw_dl[pc][t], dl);
+        load8<T>(&sm.raw_u[ubuf][pc][t], uv);
 #pragma unroll
-        for (int q2 = 0; q2 < 4; q2 += 2) {
-          const int t = tq + j + q2;
-          const float2 dl = load_pair<T>(&sm.raw_dl[cl][t]);
-          const float2 uv = load_pair<T>(&sm.raw_u[ubuf][cl][t]);
-          float2 s = __fadd2_rn(dl, make_float2(biasd, biasd));
+        for (int q2 = 0; q2 < 8; q2 += 2) {
+          float2 s = __fadd2_rn(make_float2(dl[q2], dl[q2 + 1]), make_float2(pbias, pbias));
           if (p.softplus) s = softplus2(s);
-          s.x = t < len ? s.x : 0.f;  // steps past the end leave the state alone
-          s.y = t + 1 < len ? s.y : 0.f;
-          const float2 dv = __fmul2_rn(s, uv);
-          vdt[q2] = fminf(fmaxf(s.x, -dt_clamp), dt_clamp);
-          vdt[q2 + 1] = fminf(fmaxf(s.y, -dt_clamp), dt_clamp);
+          s.x = t + q2 < len ? s.x : 0.f;  // steps past the end leave the state alone
+          s.y = t + q2 + 1 < len ? s.y : 0.f;
+          const float2 dv = __fmul2_rn(s, make_float2(uv[q2], uv[q2 + 1]));
+          vdt[q2] = fminf(fmaxf(s.x, -pclamp), pclamp);
+          vdt[q2 + 1] = fminf(fmaxf(s.y, -pclamp), pclamp);
           vdu[q2] = dv.x;
           vdu[q2 + 1] = dv.y;
         }
-        *reinterpret_cast<float4*>(&sm.dtp[cl][tq + j]) = make_float4(vdt[0], vdt[1], vdt[2], vdt[3]);
-        *reinterpret_cast<float4*>(&sm.du[cl][tq + j]) = make_float4(vdu[0], vdu[1], vdu[2], vdu[3]);
+        *reinterpret_cast<float4*>(&sm.dtp[pc][t]) = make_float4(vdt[0], vdt[1], vdt[2], vdt[3]);
+        *reinterpret_cast<float4*>(&sm.dtp[pc][t + 4]) = make_float4(vdt[4], vdt[5], vdt[6], vdt[7]);
+        *reinterpret_cast<float4*>(&sm.du[pc][t]) = make_float4(vdu[0], vdu[1], vdu[2], vdu[3]);
+        *reinterpret_cast<float4*>(&sm.du[pc][t + 4]) = make_float4(vdu[4], vdu[5], vdu[6], vdu[7]);
       }
     }
     __syncthreads();
@@ -418,12 +451,12 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
 #pragma unroll
       for (int tt = 0; tt < kSub; ++tt) {
         const int t = tb + tt;
-        const float4 bq = *reinterpret_cast<const float4*>(bf + t * kMaxN);
+        const float4 bq = *reinterpret_cast<const float4*>(bf + t * kBCRow);
         const float2 du2 = make_float2(dus[tt], dus[tt]);
         h01 = __ffma2_rn(dcur.a01[tt], h01, __fmul2_rn(du2, make_float2(bq.x, bq.y)));
         h23 = __ffma2_rn(dcur.a23[tt], h23, __fmul2_rn(du2, make_float2(bq.z, bq.w)));
         if (MODE == kFull) {
-          const float4 cq = *reinterpret_cast<const float4*>(cf + t * kMaxN);
+          const float4 cq = *reinterpret_cast<const float4*>(cf + t * kBCRow);
           float2 yv = __fmul2_rn(make_float2(cq.x, cq.y), h01);
           yv = __ffma2_rn(make_float2(cq.z, cq.w), h23, yv);
           ys[tt] = yv.x + yv.y;
