@@ -384,6 +384,46 @@ def oracle_baseline(case_host, cfg, gate, batches):
                        f"({elems} elements), float64, {cores} threads")}
 
 
+def ssd_case():
+    """Device-resident inputs of the Mamba-2 layer workload and the call that
+    runs the chunked scan on them: (config, call, tensors to keep alive)."""
+    import torch
+    from selective_state_space_08_b200 import api, synth
+    cfg = workload_cfg("mamba2_ssd")
+    sin = synth.make_ssd_inputs(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"],
+                                cfg["dstate"], cfg["dtype"], cfg["gate"], cfg["seed"], cfg["s_range"])
+    bfd = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)
+    f32d = lambda a: torch.from_numpy(a).cuda()
+    sx, sdl, sB, sC = bfd(sin["x"]), bfd(sin["delta"]), bfd(sin["B"]), bfd(sin["C"])
+    sA, sD, sbias = f32d(sin["A"]), f32d(sin["D"]), f32d(sin["delta_bias"])
+    sy = torch.empty_like(sx)
+    sh = torch.empty((cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"]),
+                     dtype=torch.float32, device="cuda")
+    sws = torch.empty(api.ssd_workspace_size(cfg["batch"], cfg["seqlen"], cfg["nheads"],
+                                             cfg["headdim"], cfg["dstate"], cfg["chunk"]),
+                      dtype=torch.uint8, device="cuda")
+    sstep = lambda: api.ssd_fwd(sx, sdl, sA, sB, sC, sD, None, sbias, True, None,
+                                chunk=cfg["chunk"], y=sy, h_last=sh, workspace=sws)
+    return cfg, sstep, (sx, sdl, sB, sC, sA, sD, sbias, sy, sh, sws)
+
+
+def run_profile(args):
+    """Runs only the product call of one workload, warmup + steps times, with
+    no timing, flush or output line: the command an ncu capture wraps
+    (select the launch with ncu's -k / -s / -c)."""
+    import torch
+    torch.cuda.set_device(0)
+    if args.profile == "scan":
+        case = ScanCase(WORKLOAD)
+        step = case.step
+    else:
+        _, step, keep = ssd_case()
+    for _ in range(args.warmup + args.steps):
+        step()
+    torch.cuda.synchronize()
+    print(f"profile: {args.warmup + args.steps} calls of the {args.profile} workload")
+
+
 def extra_workloads(steps, warmup, flush, hbm_peak):
     import torch
     from selective_state_space_08_b200 import api, synth
@@ -404,21 +444,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
         del case
         torch.cuda.empty_cache()
     # Mamba-2 chunked scan (tensor cores)
-    cfg = workload_cfg("mamba2_ssd")
-    sin = synth.make_ssd_inputs(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"],
-                                cfg["dstate"], cfg["dtype"], cfg["gate"], cfg["seed"], cfg["s_range"])
-    bfd = lambda a: torch.from_numpy(a).cuda().to(torch.bfloat16)
-    f32d = lambda a: torch.from_numpy(a).cuda()
-    sx, sdl, sB, sC = bfd(sin["x"]), bfd(sin["delta"]), bfd(sin["B"]), bfd(sin["C"])
-    sA, sD, sbias = f32d(sin["A"]), f32d(sin["D"]), f32d(sin["delta_bias"])
-    sy = torch.empty_like(sx)
-    sh = torch.empty((cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"]),
-                     dtype=torch.float32, device="cuda")
-    sws = torch.empty(api.ssd_workspace_size(cfg["batch"], cfg["seqlen"], cfg["nheads"],
-                                             cfg["headdim"], cfg["dstate"], cfg["chunk"]),
-                      dtype=torch.uint8, device="cuda")
-    sstep = lambda: api.ssd_fwd(sx, sdl, sA, sB, sC, sD, None, sbias, True, None,
-                                chunk=cfg["chunk"], y=sy, h_last=sh, workspace=sws)
+    cfg, sstep, keep = ssd_case()
     total, per, _ = time_steps(sstep, steps, warmup, flush, 1, None)
     sec = total / steps
     sb = ssd_bytes(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"])
@@ -431,8 +457,8 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
         "hbm_frac": round(sb / sec / 1e9 / hbm_peak, 4),
         "TFLOP_per_s": round(sf / sec / 1e12, 1),
         "tensor_frac_of_measured_bf16": round(sf / sec / 1e12 / bf16_peak_tflops(), 4),
-        "launches_per_call": 2}
-    del sx, sdl, sB, sC, sy, sws
+        "launches_per_call": 3}
+    del sstep, keep
     torch.cuda.empty_cache()
     # decode step on the 2.8B-layer channel count (batch 4 x 5120 channels)
     cfg = workload_cfg("mamba2p8b_layer")
@@ -564,10 +590,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the other workloads")
+    ap.add_argument("--profile", choices=["scan", "ssd"], default=None,
+                    help="only run the product call of the scan (mamba130m_layer) or\n"
+                         "chunked-scan (mamba2_ssd) workload warmup + steps times,\n"
+                         "untimed, for a profiler to capture")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.profile is not None:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
