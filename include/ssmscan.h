@@ -199,8 +199,9 @@ ssm_status_t ssm_scan_step(const ssm_step_args_t* args, ssm_stream_t stream);
  * its first int is a status word, zeroed by the call and set non-zero by the
  * GPU if a bounded wait for a tensor-core result gave up (the outputs are
  * then invalid); read it after the stream has finished.  The rest holds the
- * chunk-local states, the log-decay of every chunk and the state entering
- * every chunk.  Calls sharing a workspace must not overlap. */
+ * chunk-local states, the log-decay of every chunk, the state entering
+ * every chunk and the discretised step and cumulative log-decay of every
+ * step.  Calls sharing a workspace must not overlap. */
 typedef struct {
   int64_t batch, seqlen, nheads, headdim, dstate, chunk;
   ssm_dtype_t dtype;

@@ -1,10 +1,13 @@
 // api.cu -- host side of the libssmscan C ABI: argument checks, work planning
 // and kernel dispatch.  Every entry point is declared in include/ssmscan.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <climits>
 #include <cstdio>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -225,6 +228,64 @@ ssm_status_t run_step(const StepParams& p, bool vec4, cudaStream_t stream) {
 // ---------------------------------------------------------------------------
 constexpr size_t kSsdStatusBytes = 256;  // status word at the start of the workspace
 
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// A bf16 tensor map with 128-byte swizzle and zero fill: dims[0] is the
+// contiguous dimension, strides (bytes) are those of dims[1..rank-1].
+bool encode_bf16_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box) {
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+            const_cast<void*>(base), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The operand maps of the chunked scan (boxes of 64 elements along the
+// contiguous dimension and one chunk of steps, or 64 rows of the state).
+ssm_status_t make_ssd_maps(const SsdParams& p, SsdMaps* m) {
+  const uint64_t B = p.batch, L = p.seqlen, H = p.nheads, P = ssd::kP, N = ssd::kN;
+  const uint32_t Q = static_cast<uint32_t>(p.chunk);
+  const uint64_t xd[3] = {H * P, L, B}, xs[2] = {H * P * 2, L * H * P * 2};
+  const uint32_t xb[3] = {64, Q, 1};
+  const uint64_t bd[3] = {N, L, B}, bs[2] = {N * 2, L * N * 2};
+  const uint32_t bb[3] = {64, Q, 1};
+  const uint64_t sd[2] = {N, B * H * static_cast<uint64_t>(p.nchunks) * P}, ss[1] = {N * 2};
+  const uint32_t sb[2] = {64, 64};
+  const bool ok = encode_bf16_map(&m->x, p.x, 3, xd, xs, xb) &&
+                  encode_bf16_map(&m->B, p.B, 3, bd, bs, bb) &&
+                  encode_bf16_map(&m->C, p.C, 3, bd, bs, bb) &&
+                  encode_bf16_map(&m->sprev, p.sprev, 2, sd, ss, sb);
+  if (!ok) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "ssd: tensor-map encoding failed (driver entry point unavailable or "
+                  "operand layout rejected)");
+    return SSM_ERR_CUDA;
+  }
+  return SSM_OK;
+}
+
 ssm_status_t plan_ssd(const ssm_ssd_args_t* a, SsdParams* p, size_t* ws_bytes, bool check_ptrs) {
   if (a == nullptr) return SSM_ERR_INVALID_ARG;
   if (a->batch < 0 || a->seqlen < 0 || a->nheads < 0 || a->headdim < 0 || a->dstate < 0)
@@ -256,6 +317,10 @@ ssm_status_t plan_ssd(const ssm_ssd_args_t* a, SsdParams* p, size_t* ws_bytes, b
   p->chunk = a->chunk;
   p->nchunks = (a->seqlen + a->chunk - 1) / a->chunk;
   if (p->nchunks > 2147483647) return SSM_ERR_UNSUPPORTED;
+  // TMA coordinates are 32-bit: steps, and rows of the carried states.
+  if (a->seqlen > INT32_MAX ||
+      static_cast<double>(a->batch) * a->nheads * p->nchunks * ssd::kP > INT32_MAX)
+    return SSM_ERR_UNSUPPORTED;
   p->x = static_cast<const __nv_bfloat16*>(a->x);
   p->delta = static_cast<const __nv_bfloat16*>(a->delta);
   p->A = a->A;
@@ -271,7 +336,9 @@ ssm_status_t plan_ssd(const ssm_ssd_args_t* a, SsdParams* p, size_t* ws_bytes, b
   const size_t states = static_cast<size_t>(a->batch) * a->nheads * p->nchunks * ssd::kN * ssd::kP;
   const size_t cums = (static_cast<size_t>(a->batch) * a->nheads * p->nchunks * sizeof(float) + 255) /
                       256 * 256;
-  *ws_bytes = kSsdStatusBytes + states * sizeof(float) + cums + states * sizeof(__nv_bfloat16);
+  const size_t steps = static_cast<size_t>(a->batch) * a->nheads * p->nchunks * 2 * a->chunk;
+  *ws_bytes = kSsdStatusBytes + states * sizeof(float) + cums + states * sizeof(__nv_bfloat16) +
+              steps * sizeof(float);
   // Heads per block: the chunk-state and scan kernels run one block per SM;
   // choose the group that minimises (rounds of blocks) x (heads per block + the
   // shared C B^T product, worth about 1.5 heads).
@@ -294,7 +361,7 @@ ssm_status_t plan_ssd(const ssm_ssd_args_t* a, SsdParams* p, size_t* ws_bytes, b
 }
 
 template <int Q>
-ssm_status_t run_ssd(const SsdParams& p, cudaStream_t stream) {
+ssm_status_t run_ssd(const SsdParams& p, const SsdMaps& maps, cudaStream_t stream) {
   ssm_status_t st = SSM_OK;
   const unsigned groups = static_cast<unsigned>((p.nheads + p.hgroup - 1) / p.hgroup);
   const dim3 grid(groups, static_cast<unsigned>(p.nchunks), static_cast<unsigned>(p.batch));
@@ -303,7 +370,7 @@ ssm_status_t run_ssd(const SsdParams& p, cudaStream_t stream) {
     const size_t smem = sizeof(ssd::ChunkStateSmem<Q>) + 1024;
     st = cuda_status(set_smem(reinterpret_cast<const void*>(chunk_state), smem), "ssd: opt-in");
     if (st != SSM_OK) return st;
-    chunk_state<<<grid, ssd::kThreads, smem, stream>>>(p);
+    chunk_state<<<grid, ssd::kThreads, smem, stream>>>(p, maps);
     st = cuda_status(cudaGetLastError(), "ssd: chunk-state launch");
     if (st != SSM_OK) return st;
   }
@@ -316,12 +383,12 @@ ssm_status_t run_ssd(const SsdParams& p, cudaStream_t stream) {
     auto scan = ssd::ssd_scan_kernel<Q, true>;
     st = cuda_status(set_smem(reinterpret_cast<const void*>(scan), smem_scan), "ssd: opt-in");
     if (st != SSM_OK) return st;
-    scan<<<grid, ssd::kThreads, smem_scan, stream>>>(p);
+    scan<<<grid, ssd::kScanThreads, smem_scan, stream>>>(p, maps);
   } else {
     auto scan = ssd::ssd_scan_kernel<Q, false>;
     st = cuda_status(set_smem(reinterpret_cast<const void*>(scan), smem_scan), "ssd: opt-in");
     if (st != SSM_OK) return st;
-    scan<<<grid, ssd::kThreads, smem_scan, stream>>>(p);
+    scan<<<grid, ssd::kScanThreads, smem_scan, stream>>>(p, maps);
   }
   return cuda_status(cudaGetLastError(), "ssd: chunk scan launch");
 }
@@ -467,10 +534,18 @@ ssm_status_t ssm_scan_fwd_chunked(const ssm_ssd_args_t* args, void* workspace,
   p.sloc = reinterpret_cast<float*>(w + kSsdStatusBytes);
   p.cum_end = reinterpret_cast<float*>(w + kSsdStatusBytes + states * sizeof(float));
   p.sprev = reinterpret_cast<__nv_bfloat16*>(w + kSsdStatusBytes + states * sizeof(float) + cums);
+  p.dtc = reinterpret_cast<float*>(w + kSsdStatusBytes + states * sizeof(float) + cums +
+                                   states * sizeof(__nv_bfloat16));
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   st = cuda_status(cudaMemsetAsync(p.status, 0, sizeof(int), stream), "ssd: status reset");
   if (st != SSM_OK) return st;
-  return p.chunk == 256 ? run_ssd<256>(p, stream) : run_ssd<128>(p, stream);
+  SsdMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (p.nchunks > 0) {
+    st = make_ssd_maps(p, &maps);
+    if (st != SSM_OK) return st;
+  }
+  return p.chunk == 256 ? run_ssd<256>(p, maps, stream) : run_ssd<128>(p, maps, stream);
 }
 
 const char* ssm_status_string(ssm_status_t s) {

@@ -17,7 +17,9 @@
 // The dense contractions run as tcgen05 MMAs (bf16 operands in 128-byte-
 // swizzled shared memory, fp32 accumulators in tensor memory).  Three kernels:
 //  * ssd_chunk_state_kernel, one block per (b, chunk, head group): loads the B
-//    chunk once, then per head stages x with cp.async, scales it in place by
+//    chunk once, computes dt' and cum of every head of the group in one pass
+//    (one warp-shuffle scan per head, one block barrier for all of them) and
+//    stores them for the chunk scan, then per head stages x with cp.async, scales it in place by
 //    exp(cum_end - cum_k) dt'_k and runs S_loc^T = B^T (scaled x); two tensor-
 //    memory accumulators alternate so the next head's MMA overlaps the
 //    previous read-out.  S_loc goes to the workspace ([p][n], fp32).
@@ -26,12 +28,16 @@
 //    operand) and the final state.
 //  * ssd_scan_kernel, one block per (b, chunk, head group), the chunk in row
 //    blocks of 128 steps: G = C B^T once per group in tensor memory; per head
+//    the stored dt' and cum arrive with the head's x and S_prev (cp.async, one
+//    head ahead);
 //    the causal decay mask times dt'_k is applied per row in registers into a
 //    bf16 operand (blocks above the diagonal skipped; the block below it
 //    factorised as exp(cum_t - cum_r) exp(cum_r - cum_k) with both factors
 //    <= 1), then Y = M x and Z = C S_prev^T by MMA and the epilogue
 //    y = Y + exp(cum_t) Z + D x (optional silu(z) gate).
 #pragma once
+#include <cuda.h>  // CUtensorMap
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -55,47 +61,27 @@ struct SsdParams {
   float* sloc;           // (batch, nheads, nchunks, headdim, dstate) fp32: chunk-local states
   float* cum_end;        // (batch, nheads, nchunks): log decay over each chunk
   __nv_bfloat16* sprev;  // (batch, nheads, nchunks, headdim, dstate) bf16: state entering each chunk
+  float* dtc;            // (batch, nheads, nchunks, 2, chunk) fp32: dt', then cum, of every step
   int* status;           // bit 0: a tensor-core completion wait timed out
+};
+
+// TMA descriptors of the operands (all bf16, 128-byte swizzle, 64-element
+// boxes along the contiguous dimension, zero fill outside the tensor).
+struct SsdMaps {
+  CUtensorMap x;      // (headdim * nheads, seqlen, batch), box (64, chunk, 1)
+  CUtensorMap B;      // (dstate, seqlen, batch), box (64, chunk, 1)
+  CUtensorMap C;      // same as B
+  CUtensorMap sprev;  // (dstate, batch * nheads * nchunks * headdim), box (64, 64)
 };
 
 namespace ssd {
 
-constexpr int kThreads = 256;  // 8 warps: warps w and w + 4 share TMEM lanes 32 (w % 4)..+31
+constexpr int kThreads = 256;       // chunk-state kernel: 8 warps
+constexpr int kScanThreads = 512;   // chunk scan: 16 warps; warps w, w + 4, w + 8, w + 12
+                                    // share TMEM lanes 32 (w % 4) .. + 31
 constexpr int kN = 128;   // dstate
 constexpr int kP = 64;    // headdim
 constexpr uint32_t kWaitPolls = 1u << 22;
-
-// Block-wide inclusive prefix sum over Q values v[t] in shared memory
-// (ceil(Q / kThreads) consecutive values per thread).
-template <int Q>
-__device__ __forceinline__ void block_cumsum(float* v, float* warp_tot) {
-  constexpr int kPer = (Q + kThreads - 1) / kThreads;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float loc[kPer];
-  float run = 0.f;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int t = tid * kPer + j;
-    run += t < Q ? v[t] : 0.f;
-    loc[j] = run;
-  }
-  float incl = run;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  float off = incl - run;
-  for (int w = 0; w < warp; ++w) off += warp_tot[w];
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int t = tid * kPer + j;
-    if (t < Q) v[t] = loc[j] + off;
-  }
-  __syncthreads();
-}
 
 // The head group's dt rows for one chunk: dl[t * kMaxGroup + j] = delta[b, t0 + t, hg0 + j].
 constexpr int kMaxGroup = 24;
@@ -109,38 +95,44 @@ __device__ __forceinline__ void stage_delta(const SsdParams& p, int64_t b, int64
   }
 }
 
-// dt' and cum for head hg0 + j of the chunk (steps past the end get dt' = 0,
-// so they neither decay nor feed the state).
+// dt' and the in-chunk cumulative log decay cum of every head of the group,
+// for every step of the chunk: dtp[j * Q + t], cum[j * Q + t] (steps past the
+// end get dt' = 0, so they neither decay nor feed the state).  One step per
+// thread; one warp-shuffle scan per head, then a single block barrier before
+// the warp offsets are added.  wtot holds (kThreads / 32) x kMaxGroup floats.
 template <int Q>
-__device__ __forceinline__ void chunk_decays(const SsdParams& p, float Ah, float bias, int j,
-                                             int len, const __nv_bfloat16* dl, float* dtp,
-                                             float* cum, float* wtot) {
-  for (int i = threadIdx.x; i < Q; i += kThreads) {
+__device__ __forceinline__ void group_decays(const SsdParams& p, int64_t hg0, int nh, int len,
+                                             const __nv_bfloat16* dl, float* dtp, float* cum,
+                                             float* wtot) {
+  static_assert(Q <= kThreads, "one step per thread");
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  for (int j = 0; j < nh; ++j) {
     float s = 0.f;
-    if (i < len) {
-      s = __bfloat162float(dl[i * kMaxGroup + j]) + bias;
+    if (t < len) {
+      s = __bfloat162float(dl[t * kMaxGroup + j]) + (p.bias ? __ldg(p.bias + hg0 + j) : 0.f);
       if (p.softplus) s = softplus_f(s);
     }
-    dtp[i] = s;
-    cum[i] = s * Ah;
+    float a = s * __ldg(p.A + hg0 + j);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float n = __shfl_up_sync(0xffffffffu, a, o);
+      if (lane >= o) a += n;
+    }
+    if (t < Q) {
+      dtp[j * Q + t] = s;
+      cum[j * Q + t] = a;
+    }
+    if (lane == 31) wtot[warp * kMaxGroup + j] = a;
   }
   __syncthreads();
-  block_cumsum<Q>(cum, wtot);
-}
-
-// cp.async copy of a (rows x cols) bf16 tile, rows `ld` elements apart in
-// global memory, into 64-column blocks of 128-byte swizzled rows (block
-// stride rows * 128 bytes).  Rows >= valid are zero-filled.
-__device__ __forceinline__ void stage_tile(unsigned char* dst, const __nv_bfloat16* src, int64_t ld,
-                                           int rows, int valid, int cols) {
-  const int per_row = cols / 8;
-  for (int i = threadIdx.x; i < rows * per_row; i += kThreads) {
-    const int r = i / per_row;
-    const int c8 = (i % per_row) * 8;
-    unsigned char* d = dst + (c8 / 64) * (rows * 128) + tc::sw128_offset(r, c8 % 64);
-    const bool ok = r < valid;
-    cp_async16(d, ok ? src + r * ld + c8 : src, ok ? 16 : 0);
+  if (t < Q) {
+    for (int j = 0; j < nh; ++j) {
+      float off = 0.f;
+      for (int w = 0; w < warp; ++w) off += wtot[w * kMaxGroup + j];
+      cum[j * Q + t] += off;
+    }
   }
+  __syncthreads();
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -156,15 +148,17 @@ struct ChunkStateSmem {
   unsigned char bt[Q * kN * 2];      // B chunk: MN-major A operand of B^T (rows = time)
   unsigned char xw[2][Q * kP * 2];   // scaled x per head: MN-major B operand (rows = time)
   __nv_bfloat16 dl[Q * kMaxGroup];   // the group's delta rows
-  float cum[Q];
-  float dtp[Q];
-  float wtot[kThreads / 32];
+  float dtp[kMaxGroup * Q];          // dt' per (head of the group, step)
+  float cum[kMaxGroup * Q];          // in-chunk cumulative log decay, same layout
+  float wtot[(kThreads / 32) * kMaxGroup];
   uint64_t mbar[2];
+  uint64_t lbar[3];  // TMA completion: B chunk, x buffer 0, x buffer 1
   uint32_t tmem;
 };
 
 template <int Q>
-__global__ void __launch_bounds__(kThreads) ssd_chunk_state_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kThreads)
+    ssd_chunk_state_kernel(const SsdParams p, const __grid_constant__ SsdMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   ChunkStateSmem<Q>& sm = *reinterpret_cast<ChunkStateSmem<Q>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -176,23 +170,53 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_state_kernel(const SsdPara
   const int64_t t0 = c * Q;
   const int len = static_cast<int>(imin64(Q, L - t0));
 
+  // TMA loads: thread 0 issues them; issued[i] / waited[i] count the phases
+  // of lbar[i] (only thread 0's counts are used, to drain copies still in
+  // flight after a timed-out wait).
+  uint32_t issued[3] = {0u, 0u, 0u}, waited[3] = {0u, 0u, 0u};
+  bool ok = true;
+  auto stage_x = [&](int hj) {  // thread 0
+    uint64_t* bar = &sm.lbar[1 + (hj & 1)];
+    tc::mbar_arrive_expect_tx(bar, Q * kP * 2);
+    tc::tma_load_3d(sm.xw[hj & 1], &maps.x, static_cast<int32_t>((hg0 + hj) * kP),
+                    static_cast<int32_t>(t0), static_cast<int32_t>(b), bar);
+    ++issued[1 + (hj & 1)];
+  };
+  auto lwait = [&](int i) {
+    if (ok && !tc::mbar_wait(&sm.lbar[i], waited[i] & 1u, kWaitPolls)) ok = false;
+    if (ok) ++waited[i];
+  };
   if (warp == 0) tc::tmem_alloc(&sm.tmem, 128);
   if (tid == 0) {
     tc::mbar_init(&sm.mbar[0], 1);
     tc::mbar_init(&sm.mbar[1], 1);
+    for (int i = 0; i < 3; ++i) tc::mbar_init(&sm.lbar[i], 1);
     tc::mbar_fence_init();
+    tc::mbar_arrive_expect_tx(&sm.lbar[0], Q * kN * 2);
+    for (int hf = 0; hf < kN / 64; ++hf)
+      tc::tma_load_3d(sm.bt + hf * Q * 128, &maps.B, 64 * hf, static_cast<int32_t>(t0),
+                      static_cast<int32_t>(b), &sm.lbar[0]);
+    ++issued[0];
+    stage_x(0);
   }
-  stage_tile(sm.bt, p.B + (b * L + t0) * kN, kN, Q, len, kN);
-  stage_tile(sm.xw[0], p.x + ((b * L + t0) * H + hg0) * kP, H * kP, Q, len, kP);
-  cp_async_commit();
   stage_delta<Q>(p, b, t0, len, hg0, nh, sm.dl);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sm.tmem;
+  group_decays<Q>(p, hg0, nh, len, sm.dl, sm.dtp, sm.cum, sm.wtot);
+  // dt' and cum of every head, for the chunk scan; cum_end for the state pass
+  for (int i = tid; i < nh * Q; i += kThreads) {
+    const int j = i / Q, t = i % Q;
+    float* dst = p.dtc + ((b * H + hg0 + j) * p.nchunks + c) * (2 * Q);
+    dst[t] = sm.dtp[j * Q + t];
+    dst[Q + t] = sm.cum[j * Q + t];
+  }
+  for (int j = tid; j < nh; j += kThreads)
+    p.cum_end[(b * H + hg0 + j) * p.nchunks + c] = sm.cum[j * Q + Q - 1];
   const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
   uint32_t ph[2] = {0u, 0u};
-  bool ok = true;
+  if (tid == 0) lwait(0);  // the B chunk, read only by the MMAs
 
   auto drain = [&](int hj) {  // read out head hj's accumulator, store S_loc [p][n]
     const int bj = hj & 1;
@@ -210,19 +234,23 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_state_kernel(const SsdPara
   };
 
   for (int hi = 0; hi < nh; ++hi) {
-    const int64_t h = hg0 + hi;
     const int bi = hi & 1;
-    chunk_decays<Q>(p, p.A[h], p.bias ? p.bias[h] : 0.f, hi, len, sm.dl, sm.dtp, sm.cum, sm.wtot);
-    const float cend = sm.cum[Q - 1];
-    if (tid == 0) p.cum_end[(b * H + h) * p.nchunks + c] = cend;
-    cp_async_wait_all();  // x of this head (and, the first time, B) has landed
-    __syncthreads();
+    // Next head's x into the other buffer as soon as the MMA that last read it
+    // (head hi - 1) has completed; drain(hi - 1) waits on the same phase later.
+    if (tid == 0 && ok && hi + 1 < nh) {
+      if (hi >= 1 && !tc::mbar_wait(&sm.mbar[bi ^ 1], ph[bi ^ 1], kWaitPolls)) ok = false;
+      if (ok) stage_x(hi + 1);
+    }
+    const float* cumh = sm.cum + hi * Q;
+    const float* dtph = sm.dtp + hi * Q;
+    const float cend = cumh[Q - 1];
+    lwait(1 + bi);  // x of this head has landed
     // scale x rows in place: w_t = exp(cum_end - cum_t) dt'_t
     for (int i = tid; i < Q * (kP / 8); i += kThreads) {
       const int t = i / (kP / 8);
       const int p8 = (i % (kP / 8)) * 8;
       uint4* ptr = reinterpret_cast<uint4*>(sm.xw[bi] + tc::sw128_offset(t, p8));
-      const float w = ex2_approx((cend - sm.cum[t]) * kLog2e) * sm.dtp[t];
+      const float w = ex2_approx((cend - cumh[t]) * kLog2e) * dtph[t];
       uint4 v = *ptr;
       uint32_t* vw = &v.x;
 #pragma unroll
@@ -243,14 +271,14 @@ __global__ void __launch_bounds__(kThreads) ssd_chunk_state_kernel(const SsdPara
                      tc::make_sdesc(x0 + ks * 2048, Q * 128, 1024), idesc, ks > 0);
       tc::mma_commit(&sm.mbar[bi]);
     }
-    if (hi >= 1) drain(hi - 1);  // frees xw[bi ^ 1]
-    if (hi + 1 < nh) {
-      stage_tile(sm.xw[bi ^ 1], p.x + ((b * L + t0) * H + h + 1) * kP, H * kP, Q, len, kP);
-      cp_async_commit();
-    }
+    if (hi >= 1) drain(hi - 1);
   }
   if (nh > 0) drain(nh - 1);
-  if (!ok && tid == 0) atomicOr(p.status, 1);
+  if (!ok && tid == 0) {
+    atomicOr(p.status, 1);
+    for (int i = 0; i < 3; ++i)  // copies still in flight land before the block exits
+      for (; waited[i] < issued[i]; ++waited[i]) tc::mbar_wait(&sm.lbar[i], waited[i] & 1u, kWaitPolls);
+  }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 128);
@@ -298,18 +326,17 @@ struct ScanSmem {
   unsigned char x0[Q * kP * 2];   // even heads' x: MN-major B operand (rows = time)
   unsigned char sp0[kP * kN * 2]; // even heads' S_prev [p][n]: K-major B operand (rows = p)
   unsigned char m[128 * 128 * 2]; // masked decays, K-major A operand: two 64-key halves
-  float cum[Q];
-  float dtp[Q];
+  float dc[2][2 * Q];             // per head (two buffers): dt'[Q], then cum[Q]
   float vk[128];                  // exp(cum_r - cum_k) dt'_k below the diagonal block
-  __nv_bfloat16 dl[Q * kMaxGroup]; // the group's delta rows
-  float hA[kMaxGroup], hbias[kMaxGroup], hD[kMaxGroup];
-  float wtot[kThreads / 32];
+  float hD[kMaxGroup];
   uint64_t mbar[2];
+  uint64_t lbar[3];  // TMA completion: C and B chunks, head buffers 0 and 1
   uint32_t tmem;
 };
 
 template <int Q, bool HAS_Z>
-__global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
+__global__ void __launch_bounds__(kScanThreads, 1)
+    ssd_scan_kernel(const SsdParams p, const __grid_constant__ SsdMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   ScanSmem<Q>& sm = *reinterpret_cast<ScanSmem<Q>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -325,41 +352,54 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
   constexpr uint32_t kColY = 384, kColZ = 448;
   unsigned char* xbuf[2] = {sm.x0, sm.bk};
   unsigned char* spbuf[2] = {sm.sp0, sm.bk + Q * kP * 2};
-  auto stage_head = [&](int hj) {
+  // TMA loads: thread 0 issues them; issued[i] / waited[i] count the phases
+  // of lbar[i] (thread 0's counts drain copies still in flight after a
+  // timed-out wait).
+  uint32_t issued[3] = {0u, 0u, 0u}, waited[3] = {0u, 0u, 0u};
+  bool ok = true;
+  auto stage_head = [&](int hj) {  // thread 0: x, S_prev, dt' and cum of head hg0 + hj
     const int64_t h = hg0 + hj;
-    stage_tile(xbuf[hj & 1], p.x + ((b * L + t0) * H + h) * kP, H * kP, Q, len, kP);
-    stage_tile(spbuf[hj & 1], p.sprev + ((b * H + h) * p.nchunks + c) * kP * kN, kN, kP, kP, kN);
-    cp_async_commit();
+    uint64_t* bar = &sm.lbar[1 + (hj & 1)];
+    tc::mbar_arrive_expect_tx(bar, Q * kP * 2 + kP * kN * 2 + 2 * Q * 4);
+    tc::tma_load_3d(xbuf[hj & 1], &maps.x, static_cast<int32_t>(h * kP), static_cast<int32_t>(t0),
+                    static_cast<int32_t>(b), bar);
+    const int32_t row = static_cast<int32_t>(((b * H + h) * p.nchunks + c) * kP);
+    for (int hf = 0; hf < kN / 64; ++hf)
+      tc::tma_load_2d(spbuf[hj & 1] + hf * kP * 128, &maps.sprev, 64 * hf, row, bar);
+    tc::bulk_load(sm.dc[hj & 1], p.dtc + ((b * H + h) * p.nchunks + c) * (2 * Q), 2 * Q * 4, bar);
+    ++issued[1 + (hj & 1)];
+  };
+  auto lwait = [&](int i) {
+    if (ok && !tc::mbar_wait(&sm.lbar[i], waited[i] & 1u, kWaitPolls)) ok = false;
+    if (ok) ++waited[i];
   };
 
   if (warp == 0) tc::tmem_alloc(&sm.tmem, 512);
   if (tid == 0) {
     tc::mbar_init(&sm.mbar[0], 1);
     tc::mbar_init(&sm.mbar[1], 1);
+    for (int i = 0; i < 3; ++i) tc::mbar_init(&sm.lbar[i], 1);
     tc::mbar_fence_init();
+    tc::mbar_arrive_expect_tx(&sm.lbar[0], 2 * Q * kN * 2);
+    for (int hf = 0; hf < kN / 64; ++hf) {
+      tc::tma_load_3d(sm.c + hf * Q * 128, &maps.C, 64 * hf, static_cast<int32_t>(t0),
+                      static_cast<int32_t>(b), &sm.lbar[0]);
+      tc::tma_load_3d(sm.bk + hf * Q * 128, &maps.B, 64 * hf, static_cast<int32_t>(t0),
+                      static_cast<int32_t>(b), &sm.lbar[0]);
+    }
+    ++issued[0];
+    stage_head(0);
   }
-  stage_tile(sm.c, p.C + (b * L + t0) * kN, kN, Q, len, kN);
-  stage_tile(sm.bk, p.B + (b * L + t0) * kN, kN, Q, len, kN);
-  cp_async_commit();
-  stage_head(0);
-  stage_delta<Q>(p, b, t0, len, hg0, nh, sm.dl);
-  for (int j = tid; j < nh; j += kThreads) {
-    sm.hA[j] = p.A[hg0 + j];
-    sm.hbias[j] = p.bias ? p.bias[hg0 + j] : 0.f;
-    sm.hD[j] = p.D ? p.D[hg0 + j] : 0.f;
-  }
-  cp_async_wait_all();
-  tc::fence_proxy_async_smem();
+  for (int j = tid; j < nh; j += kScanThreads) sm.hD[j] = p.D ? p.D[hg0 + j] : 0.f;
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = sm.tmem;
   const int quarter = warp & 3;         // TMEM lanes 32 quarter ..+31 = rows of the row block
-  const int chalf = warp >> 2;          // which 32 of each 64 columns this warp handles
+  const int cq = warp >> 2;             // which 16 of each 64 columns this warp handles
   const int rl = 32 * quarter + (tid & 31);  // this thread's row within the row block
   const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
   uint32_t ph[2] = {0u, 0u};
-  bool ok = true;
   auto wait_bar = [&](int i) {
     if (ok && !tc::mbar_wait(&sm.mbar[i], ph[i], kWaitPolls)) ok = false;
     ph[i] ^= 1;
@@ -367,7 +407,8 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
   };
 
   // G = C B^T for the chunk, shared by every head of the group.
-  if (tid == 0) {
+  if (tid == 0) lwait(0);  // C and B chunks landed (read only by the MMAs)
+  if (tid == 0 && ok) {
     const uint32_t ca = tc::smem_u32(sm.c), bb = tc::smem_u32(sm.bk);
 #pragma unroll
     for (int ks = 0; ks < kN / 16; ++ks) {
@@ -385,27 +426,26 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
   for (int hi = 0; hi < nh; ++hi) {
     const int64_t h = hg0 + hi;
     const int bi = hi & 1;
-    if (hi + 1 < nh) stage_head(hi + 1);  // into the other buffers (their last use has completed)
-    chunk_decays<Q>(p, sm.hA[hi], sm.hbias[hi], hi, len, sm.dl, sm.dtp, sm.cum, sm.wtot);
-    if (Q == 256) {  // factor below the diagonal block: reference step r = 127
-      const float cr = sm.cum[127];
-      for (int k = tid; k < 128; k += kThreads)
-        sm.vk[k] = ex2_approx((cr - sm.cum[k]) * kLog2e) * sm.dtp[k];
+    // into the other buffers: their last readers finished before the barrier
+    // that ended the previous head
+    if (tid == 0 && ok && hi + 1 < nh) stage_head(hi + 1);
+    lwait(1 + bi);  // this head's operands landed
+    const float* dtph = sm.dc[bi];
+    const float* cumh = sm.dc[bi] + Q;
+    // Factor below the diagonal block (reference step r = 127).  Row block 1
+    // reads it only after row block 0's barriers.
+    if (Q == 256) {
+      const float cr = cumh[127];
+      for (int k = tid; k < 128; k += kScanThreads)
+        sm.vk[k] = ex2_approx((cr - cumh[k]) * kLog2e) * dtph[k];
     }
-    if (hi + 1 < nh) {
-      asm volatile("cp.async.wait_group 1;\n" ::: "memory");  // this head's x / S_prev landed
-    } else {
-      cp_async_wait_all();
-    }
-    tc::fence_proxy_async_smem();
-    __syncthreads();
     const uint32_t xb = tc::smem_u32(xbuf[bi]);
     const uint32_t spb = tc::smem_u32(spbuf[bi]);
     const float Dh = sm.hD[hi];
 
     for (int i = 0; i < Q / 128; ++i) {
       const int tr = 128 * i + rl;  // this thread's row (step) in the chunk
-      const float cum_t = sm.cum[tr];
+      const float cum_t = cumh[tr];
       const uint32_t gcol = i == 0 ? kColG0 : kColG1;
       // Z_i = C_i S_prev^T (K = states)
       if (tid == 0 && ok) {
@@ -417,49 +457,49 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
         }
       }
       // Y_i = sum over key blocks of (masked decays) x, 64 keys per step.  Each
-      // warp handles 32 keys of a block; the next block's G slab is loaded from
+      // warp handles 16 keys of a block; the next block's G slab is loaded from
       // tensor memory while the current one is turned into decays.
       const int nkb = 2 * (i + 1);  // 64-key blocks reaching this row block
       auto slab_active = [&](int kb) {  // warp-uniform: skip slabs above the diagonal
-        return kb < 2 * i || (64 * kb + 32 * chalf - 128 * i) <= 32 * quarter + 31;
+        return kb < 2 * i || (64 * kb + 16 * cq - 128 * i) <= 32 * quarter + 31;
       };
-      uint32_t gA[32], gB[32];  // double buffer of G slabs (named, so they stay in registers)
-      if (slab_active(0)) tc::tmem_ld32_issue(tmem + lane_off + gcol + 32 * chalf, gA);
-      auto key_block = [&](int kb, const uint32_t (&cur_raw)[32], uint32_t (&next_raw)[32]) {
+      uint32_t gA[16], gB[16];  // double buffer of G slabs (named, so they stay in registers)
+      if (slab_active(0)) tc::tmem_ld16_issue(tmem + lane_off + gcol + 16 * cq, gA);
+      auto key_block = [&](int kb, const uint32_t (&cur_raw)[16], uint32_t (&next_raw)[16]) {
         const int mb = kb & 1;  // shared-memory half of m used by this key block
         const bool active = slab_active(kb);
         tc::tmem_wait();
-        uint32_t cur[32];
+        uint32_t cur[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) cur[j] = cur_raw[j];
+        for (int j = 0; j < 16; ++j) cur[j] = cur_raw[j];
         if (kb + 1 < nkb && slab_active(kb + 1))
-          tc::tmem_ld32_issue(tmem + lane_off + gcol + 64 * (kb + 1) + 32 * chalf, next_raw);
+          tc::tmem_ld16_issue(tmem + lane_off + gcol + 64 * (kb + 1) + 16 * cq, next_raw);
         if (kb >= 2) wait_bar(mb);  // the MMA that read this half two steps ago is done
         const bool below = i == 1 && kb < 2;          // keys 0..127 of rows 128..255
         const int kbase = 64 * kb;
-        const int cb = 32 * chalf;
+        const int cb = 16 * cq;
         const int k0 = kbase + cb;
-        uint32_t packed[16];
+        uint32_t packed[8];
         if (active) {
           if (below) {
-            const float urow = ex2_approx((cum_t - sm.cum[127]) * kLog2e);
-            float vv[32];
+            const float urow = ex2_approx((cum_t - cumh[127]) * kLog2e);
+            float vv[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
+            for (int j = 0; j < 16; j += 4)
               *reinterpret_cast<float4*>(&vv[j]) = *reinterpret_cast<const float4*>(&sm.vk[k0 + j]);
 #pragma unroll
-            for (int j = 0; j < 32; j += 2)
+            for (int j = 0; j < 16; j += 2)
               packed[j / 2] = pack_bf16(__uint_as_float(cur[j]) * urow * vv[j],
                                         __uint_as_float(cur[j + 1]) * urow * vv[j + 1]);
           } else {
-            float ck[32], dk[32];
+            float ck[16], dk[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              *reinterpret_cast<float4*>(&ck[j]) = *reinterpret_cast<const float4*>(&sm.cum[k0 + j]);
-              *reinterpret_cast<float4*>(&dk[j]) = *reinterpret_cast<const float4*>(&sm.dtp[k0 + j]);
+            for (int j = 0; j < 16; j += 4) {
+              *reinterpret_cast<float4*>(&ck[j]) = *reinterpret_cast<const float4*>(&cumh[k0 + j]);
+              *reinterpret_cast<float4*>(&dk[j]) = *reinterpret_cast<const float4*>(&dtph[k0 + j]);
             }
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
+            for (int j = 0; j < 16; j += 2) {
               const int k = k0 + j;
               const float e0 = k <= tr ? ex2_approx((cum_t - ck[j]) * kLog2e) * dk[j] * __uint_as_float(cur[j]) : 0.f;
               const float e1 = k + 1 <= tr ? ex2_approx((cum_t - ck[j + 1]) * kLog2e) * dk[j + 1] * __uint_as_float(cur[j + 1]) : 0.f;
@@ -468,10 +508,10 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) packed[j] = 0u;
+          for (int j = 0; j < 8; ++j) packed[j] = 0u;
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           *reinterpret_cast<uint4*>(sm.m + mb * (128 * 128) + tc::sw128_offset(rl, cb + 8 * q)) =
               make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         }
@@ -504,39 +544,35 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
       const float ec = ex2_approx(cum_t * kLog2e);
       const int64_t row = ((b * L + t0 + (row_ok ? tr : 0)) * H + h) * kP;
       {
-        const int cb = 32 * chalf;
-        uint32_t yr[32], zr32[32];
-        tc::tmem_ld32_issue(tmem + lane_off + kColY + cb, yr);
-        tc::tmem_ld32_issue(tmem + lane_off + kColZ + cb, zr32);
+        const int cb = 16 * cq;
+        uint32_t yr[16], zr16[16];
+        tc::tmem_ld16_issue(tmem + lane_off + kColY + cb, yr);
+        tc::tmem_ld16_issue(tmem + lane_off + kColZ + cb, zr16);
         tc::tmem_wait();
-        float yv[32], zv[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          yv[j] = __uint_as_float(yr[j]);
-          zv[j] = __uint_as_float(zr32[j]);
-        }
         if (row_ok) {
 #pragma unroll
-        for (int q = 0; q < 32; q += 8) {
-          const uint4 xr = *reinterpret_cast<const uint4*>(xbuf[bi] + tc::sw128_offset(tr, cb + q));
-          const uint32_t* xw = &xr.x;
-          uint4 zr = make_uint4(0, 0, 0, 0);
-          if (HAS_Z) zr = *reinterpret_cast<const uint4*>(p.z + row + cb + q);
-          const uint32_t* zw = &zr.x;
-          uint4 o;
-          uint32_t* ow = &o.x;
+          for (int q = 0; q < 16; q += 8) {
+            const uint4 xr = *reinterpret_cast<const uint4*>(xbuf[bi] + tc::sw128_offset(tr, cb + q));
+            const uint32_t* xw = &xr.x;
+            uint4 zr = make_uint4(0, 0, 0, 0);
+            if (HAS_Z) zr = *reinterpret_cast<const uint4*>(p.z + row + cb + q);
+            const uint32_t* zw = &zr.x;
+            uint4 o;
+            uint32_t* ow = &o.x;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float v0 = yv[q + 2 * j] + ec * zv[q + 2 * j] + Dh * __uint_as_float(xw[j] << 16);
-            float v1 = yv[q + 2 * j + 1] + ec * zv[q + 2 * j + 1] + Dh * __uint_as_float(xw[j] & 0xffff0000u);
-            if (HAS_Z) {
-              v0 *= silu_f(__uint_as_float(zw[j] << 16));
-              v1 *= silu_f(__uint_as_float(zw[j] & 0xffff0000u));
+            for (int j = 0; j < 4; ++j) {
+              float v0 = __uint_as_float(yr[q + 2 * j]) + ec * __uint_as_float(zr16[q + 2 * j]) +
+                         Dh * __uint_as_float(xw[j] << 16);
+              float v1 = __uint_as_float(yr[q + 2 * j + 1]) + ec * __uint_as_float(zr16[q + 2 * j + 1]) +
+                         Dh * __uint_as_float(xw[j] & 0xffff0000u);
+              if (HAS_Z) {
+                v0 *= silu_f(__uint_as_float(zw[j] << 16));
+                v1 *= silu_f(__uint_as_float(zw[j] & 0xffff0000u));
+              }
+              ow[j] = pack_bf16(v0, v1);
             }
-            ow[j] = pack_bf16(v0, v1);
+            *reinterpret_cast<uint4*>(p.y + row + cb + q) = o;
           }
-          *reinterpret_cast<uint4*>(p.y + row + cb + q) = o;
-        }
         }
       }
       tc::fence_before_sync();
@@ -544,7 +580,11 @@ __global__ void __launch_bounds__(kThreads) ssd_scan_kernel(const SsdParams p) {
       tc::fence_after_sync();
     }
   }
-  if (!ok && tid == 0) atomicOr(p.status, 1);
+  if (!ok && tid == 0) {
+    atomicOr(p.status, 1);
+    for (int i = 0; i < 3; ++i)  // copies still in flight land before the block exits
+      for (; waited[i] < issued[i]; ++waited[i]) tc::mbar_wait(&sm.lbar[i], waited[i] & 1u, kWaitPolls);
+  }
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
