@@ -77,8 +77,11 @@ struct SsdMaps {
 namespace ssd {
 
 constexpr int kThreads = 256;       // chunk-state kernel: 8 warps
-constexpr int kScanThreads = 512;   // chunk scan: 16 warps; warps w, w + 4, w + 8, w + 12
-                                    // share TMEM lanes 32 (w % 4) .. + 31
+// Chunk scan: 16 compute warps (warps w, w + 4, w + 8, w + 12 share TMEM
+// lanes 32 (w % 4) .. + 31) and one producer warp whose first thread issues
+// every TMA load and MMA, so no compute warp waits behind MMA issue.
+constexpr int kScanCompute = 512;
+constexpr int kScanThreads = kScanCompute + 32;
 constexpr int kN = 128;   // dstate
 constexpr int kP = 64;    // headdim
 constexpr uint32_t kWaitPolls = 1u << 22;
@@ -341,6 +344,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   ScanSmem<Q>& sm = *reinterpret_cast<ScanSmem<Q>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5;
+  const bool producer = tid >= kScanCompute;      // the producer warp
+  const bool issuer = tid == kScanCompute;        // its thread that issues TMA and MMA
   const int64_t hg0 = static_cast<int64_t>(blockIdx.x) * p.hgroup;
   const int64_t c = blockIdx.y, b = blockIdx.z;
   const int64_t L = p.seqlen, H = p.nheads;
@@ -352,12 +357,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   constexpr uint32_t kColY = 384, kColZ = 448;
   unsigned char* xbuf[2] = {sm.x0, sm.bk};
   unsigned char* spbuf[2] = {sm.sp0, sm.bk + Q * kP * 2};
-  // TMA loads: thread 0 issues them; issued[i] / waited[i] count the phases
-  // of lbar[i] (thread 0's counts drain copies still in flight after a
+  // TMA loads: the issuer thread issues them; issued[i] / waited[i] count the
+  // phases of lbar[i] (its counts drain copies still in flight after a
   // timed-out wait).
   uint32_t issued[3] = {0u, 0u, 0u}, waited[3] = {0u, 0u, 0u};
   bool ok = true;
-  auto stage_head = [&](int hj) {  // thread 0: x, S_prev, dt' and cum of head hg0 + hj
+  auto stage_head = [&](int hj) {  // issuer: x, S_prev, dt' and cum of head hg0 + hj
     const int64_t h = hg0 + hj;
     uint64_t* bar = &sm.lbar[1 + (hj & 1)];
     tc::mbar_arrive_expect_tx(bar, Q * kP * 2 + kP * kN * 2 + 2 * Q * 4);
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   };
 
   if (warp == 0) tc::tmem_alloc(&sm.tmem, 512);
-  if (tid == 0) {
+  if (issuer) {
     tc::mbar_init(&sm.mbar[0], 1);
     tc::mbar_init(&sm.mbar[1], 1);
     for (int i = 0; i < 3; ++i) tc::mbar_init(&sm.lbar[i], 1);
@@ -407,8 +412,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   };
 
   // G = C B^T for the chunk, shared by every head of the group.
-  if (tid == 0) lwait(0);  // C and B chunks landed (read only by the MMAs)
-  if (tid == 0 && ok) {
+  if (issuer) lwait(0);  // C and B chunks landed (read only by the MMAs)
+  if (issuer && ok) {
     const uint32_t ca = tc::smem_u32(sm.c), bb = tc::smem_u32(sm.bk);
 #pragma unroll
     for (int ks = 0; ks < kN / 16; ++ks) {
@@ -421,14 +426,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
     tc::mma_commit(&sm.mbar[0]);
   }
-  wait_bar(0);  // the B chunk's region is free from here on
+  wait_bar(0);  // the B chunk's region is free from here on (the producer warp
+                // waits on no MMA after this one: the barriers order it)
 
   for (int hi = 0; hi < nh; ++hi) {
     const int64_t h = hg0 + hi;
     const int bi = hi & 1;
     // into the other buffers: their last readers finished before the barrier
     // that ended the previous head
-    if (tid == 0 && ok && hi + 1 < nh) stage_head(hi + 1);
+    if (issuer && ok && hi + 1 < nh) stage_head(hi + 1);
     lwait(1 + bi);  // this head's operands landed
     const float* dtph = sm.dc[bi];
     const float* cumh = sm.dc[bi] + Q;
@@ -448,7 +454,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       const float cum_t = cumh[tr];
       const uint32_t gcol = i == 0 ? kColG0 : kColG1;
       // Z_i = C_i S_prev^T (K = states)
-      if (tid == 0 && ok) {
+      if (issuer && ok) {
         const uint32_t ca = tc::smem_u32(sm.c) + i * 128 * 128;
         for (int ks = 0; ks < kN / 16; ++ks) {
           tc::mma_bf16(tmem + kColZ, tc::make_sdesc(ca + (ks / 4) * (Q * 128) + (ks % 4) * 32, 16, 1024),
@@ -464,9 +470,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         return kb < 2 * i || (64 * kb + 16 * cq - 128 * i) <= 32 * quarter + 31;
       };
       uint32_t gA[16], gB[16];  // double buffer of G slabs (named, so they stay in registers)
-      if (slab_active(0)) tc::tmem_ld16_issue(tmem + lane_off + gcol + 16 * cq, gA);
+      if (!producer && slab_active(0)) tc::tmem_ld16_issue(tmem + lane_off + gcol + 16 * cq, gA);
       auto key_block = [&](int kb, const uint32_t (&cur_raw)[16], uint32_t (&next_raw)[16]) {
         const int mb = kb & 1;  // shared-memory half of m used by this key block
+        const int kbase = 64 * kb;
+        if (!producer) {
         const bool active = slab_active(kb);
         tc::tmem_wait();
         uint32_t cur[16];
@@ -476,7 +484,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tc::tmem_ld16_issue(tmem + lane_off + gcol + 64 * (kb + 1) + 16 * cq, next_raw);
         if (kb >= 2) wait_bar(mb);  // the MMA that read this half two steps ago is done
         const bool below = i == 1 && kb < 2;          // keys 0..127 of rows 128..255
-        const int kbase = 64 * kb;
         const int cb = 16 * cq;
         const int k0 = kbase + cb;
         uint32_t packed[8];
@@ -516,10 +523,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         }
         tc::fence_proxy_async_smem();
+        }
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        if (tid == 0 && ok) {
+        if (issuer && ok) {
           const uint32_t ma = tc::smem_u32(sm.m) + mb * (128 * 128);
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
@@ -535,15 +543,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         key_block(kb + 1, gB, gA);
       }
       // both halves' last MMAs (this row block's Y and Z) complete
-      wait_bar(0);
-      wait_bar(1);
+      if (!producer) {
+        wait_bar(0);
+        wait_bar(1);
+      }
 
       // epilogue: y = Y + exp(cum_t) Z + D x (then the gate), row tr.  The
       // tensor-memory loads are warp-collective: every lane runs them.
       const bool row_ok = tr < len;
       const float ec = ex2_approx(cum_t * kLog2e);
       const int64_t row = ((b * L + t0 + (row_ok ? tr : 0)) * H + h) * kP;
-      {
+      if (!producer) {
         const int cb = 16 * cq;
         uint32_t yr[16], zr16[16];
         tc::tmem_ld16_issue(tmem + lane_off + kColY + cb, yr);
@@ -580,8 +590,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       tc::fence_after_sync();
     }
   }
-  if (!ok && tid == 0) {
-    atomicOr(p.status, 1);
+  if (!ok) atomicOr(p.status, 1);
+  if (!ok && issuer) {
     for (int i = 0; i < 3; ++i)  // copies still in flight land before the block exits
       for (; waited[i] < issued[i]; ++waited[i]) tc::mbar_wait(&sm.lbar[i], waited[i] & 1u, kWaitPolls);
   }
