@@ -314,10 +314,12 @@ def time_steps(step, steps, warmup, flush, world, device, sampler_index=None):
     return total, per, sampler.record()
 
 
-def e2e_measure(case, steps, warmup):
-    """The same metric through the C ABI from pinned host buffers: per step the
-    host->device copies of every input, the scan, and the device->host copies
-    of y and h_last, all inside the timed region."""
+def e2e_measure(case, steps, warmup, slice_batch=1):
+    """The same metric through the C ABI from page-locked host buffers
+    (ssm_scan_fwd_host): per step the host->device copies of every input, the
+    scan and the device->host copies of y and h_last, all inside the timed
+    region.  The call pipelines batch slices of ``slice_batch`` sequences, so
+    the copies in both directions overlap each other and the scans."""
     import numpy as np
     import torch
     from selective_state_space_08_b200 import api
@@ -325,18 +327,16 @@ def e2e_measure(case, steps, warmup):
     pinned = {k: case.t[k].cpu().pin_memory() for k in names if case.t[k] is not None}
     y_host = torch.empty(case.y.shape, dtype=case.y.dtype).pin_memory()
     h_host = torch.empty(case.h.shape, dtype=torch.float32).pin_memory()
-    dev = {k: torch.empty_like(case.t[k]) for k in pinned}
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = y_host.numel() * y_host.element_size() + h_host.numel() * 4
+    args = [pinned["u"], pinned["delta"], pinned["A"], pinned["B"], pinned["C"], pinned.get("D"),
+            pinned.get("z"), pinned.get("delta_bias"), True, None]
+    staging = torch.empty(api.scan_fwd_host_staging_size(*args, slice_batch=slice_batch),
+                          dtype=torch.uint8, device="cuda")
 
     def one():
-        for k, v in pinned.items():
-            dev[k].copy_(v, non_blocking=True)
-        api.scan_fwd(dev["u"], dev["delta"], dev["A"], dev["B"], dev["C"], dev.get("D"),
-                     dev.get("z"), dev.get("delta_bias"), True, None, y=case.y, h_last=case.h,
-                     workspace=case.ws)
-        y_host.copy_(case.y, non_blocking=True)
-        h_host.copy_(case.h, non_blocking=True)
+        api.scan_fwd_host(*args, y=y_host, h_last=h_host, slice_batch=slice_batch,
+                          staging=staging, synchronize=False)
 
     for _ in range(warmup):
         one()
@@ -351,7 +351,8 @@ def e2e_measure(case, steps, warmup):
     assert bool(np.isfinite(y_host.float().numpy()).all())
     return {"value": round(case.bytes / sec / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": round(sec * 1e3, 4)}
+            "ms_per_step": round(sec * 1e3, 4), "api": "ssm_scan_fwd_host",
+            "slice_batch": slice_batch}
 
 
 def oracle_baseline(case_host, cfg, gate, batches):

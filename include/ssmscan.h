@@ -148,6 +148,32 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t w
  *    and must be serialised by the caller. */
 ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_args_t* args, ssm_stream_t stream);
 
+/* The selective scan on inputs and outputs in HOST memory, for callers whose
+ * data live on the host.  The pages have no counterpart to this entry point:
+ * it is a packaging of ssm_scan_fwd that hides the PCIe transfers behind one
+ * another.  The batch is cut into slices of `slice_batch` sequences that move
+ * through two slots of device staging: while slice s is scanned on `stream`,
+ * slice s + 1 is copied in and slice s - 1 copied out, on two copy streams
+ * that the library creates on the first call on each device and keeps.
+ *
+ * Arguments: those of ssm_scan_fwd, except that every pointer in `args` is a
+ * HOST pointer and only the default contiguous layouts are accepted (every
+ * stride 0; others return SSM_ERR_UNSUPPORTED).  Page-locked host memory
+ * (cudaHostAlloc or cudaHostRegister) lets the copies overlap; pageable
+ * memory gives the same results without the overlap.  slice_batch >= 1.
+ * `staging`: device memory, 256-byte aligned, at least
+ * ssm_scan_fwd_host_staging_size(args, slice_batch) bytes, contents ignored
+ * (SSM_ERR_WORKSPACE if missing or smaller).
+ * Ordering: the copies start after the work queued on `stream` before the
+ * call, and `stream` waits for the last copy back, so y and h_last on the
+ * host are complete once `stream` has finished; until then the host buffers
+ * and the staging must not be touched.  The call only queues work.  Calls
+ * that share a staging buffer must not overlap.  On an error return part of
+ * the work may already be queued and the outputs are undefined. */
+size_t ssm_scan_fwd_host_staging_size(const ssm_scan_args_t* args, int64_t slice_batch);
+ssm_status_t ssm_scan_fwd_host(const ssm_scan_args_t* args, int64_t slice_batch, void* staging,
+                               size_t staging_bytes, ssm_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * One decode step ("Mamba与选择性SSM", section 5.4): the scan above for a
  * single time step, with the state read and overwritten in place.

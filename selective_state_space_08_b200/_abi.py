@@ -75,6 +75,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_scan_fwd.restype = ctypes.c_int
     lib.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _vp]
     lib.ssm_scan_fwd_noalloc.restype = ctypes.c_int
+    lib.ssm_scan_fwd_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), _i64]
+    lib.ssm_scan_fwd_host_staging_size.restype = ctypes.c_size_t
+    lib.ssm_scan_fwd_host.argtypes = [ctypes.POINTER(ScanArgs), _i64, _vp, ctypes.c_size_t, _vp]
+    lib.ssm_scan_fwd_host.restype = ctypes.c_int
     lib.ssm_scan_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
     lib.ssm_scan_step.restype = ctypes.c_int
     lib.ssm_scan_fwd_chunked_workspace_size.argtypes = [ctypes.POINTER(SsdArgs)]

@@ -37,6 +37,18 @@ def _cuda(name, t, dtype=None, dims=None):
     return t
 
 
+def _host(name, t, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise ValueError(f"{name} must be a CPU tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
 def _seq_strides(name, t):
     """(batch stride, row stride) of a (batch, rows, L) tensor with unit stride along L."""
     if t.shape[-1] > 1 and t.stride(-1) != 1:
@@ -44,7 +56,10 @@ def _seq_strides(name, t):
     return (t.stride(0), t.stride(1))
 
 
-def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last):
+def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last, host=False):
+    """ScanArgs for device tensors, or (host=True) for contiguous CPU tensors,
+    whose strides are left at 0 (the contiguous default)."""
+    check = _host if host else _cuda
     dt = u.dtype
     if dt not in _DT:
         raise ValueError("u must be float32 or bfloat16")
@@ -59,7 +74,7 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_las
     for name, t, shape in (("A", A, (dim, N)), ("D", D, (dim,)), ("delta_bias", delta_bias, (dim,)),
                            ("h0", h0, (batch, dim, N)), ("h_last", h_last, (batch, dim, N))):
         if t is not None:
-            _cuda(name, t, torch.float32)
+            check(name, t, torch.float32)
             if tuple(t.shape) != shape or not t.is_contiguous():
                 raise ValueError(f"{name} must be contiguous float32 of shape {shape}")
     a = _abi.ScanArgs()
@@ -71,7 +86,7 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_las
     a.h0, a.y, a.h_last = _ptr(h0), _ptr(y), _ptr(h_last)
     for field, name, t in (("u_stride", "u", u), ("delta_stride", "delta", delta), ("z_stride", "z", z),
                            ("y_stride", "y", y), ("B_stride", "B", B), ("C_stride", "C", C)):
-        if t is not None:
+        if t is not None and not host:
             sb, sr = _seq_strides(name, t)
             getattr(a, field)[0] = sb
             getattr(a, field)[1] = sr
@@ -131,6 +146,61 @@ def scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_s
     a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last)
     _abi.check(_abi.load().ssm_scan_fwd_noalloc(ctypes.byref(a), _stream(stream)),
                "ssm_scan_fwd_noalloc")
+    return y, h_last
+
+
+def scan_fwd_host_staging_size(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                               delta_softplus=True, h0=None, *, slice_batch=1,
+                               return_last_state=True) -> int:
+    """Bytes of device staging ``scan_fwd_host`` needs for these CPU tensors."""
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0)):
+        _host(name, t)
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, None, None, host=True)
+    # The outputs' presence (not their address) enters the size: stand-ins.
+    a.y = ctypes.c_void_p(4096)
+    if return_last_state:
+        a.h_last = ctypes.c_void_p(4096)
+    n = _abi.load().ssm_scan_fwd_host_staging_size(ctypes.byref(a), int(slice_batch))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    return int(n)
+
+
+def scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+                  h0=None, *, y=None, h_last=None, return_last_state=True, slice_batch=1,
+                  staging=None, stream=None, synchronize=True):
+    """Selective scan on contiguous CPU tensors (page-locked ones let the
+    copies overlap): the batch moves through device staging in slices of
+    ``slice_batch`` sequences, copies in, scans and copies out overlapping.
+    Outputs are CPU tensors (page-locked when allocated here); with
+    ``synchronize=False`` they are complete only once ``stream`` (default:
+    the current torch stream) has finished.  Returns (y, h_last)."""
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+        _host(name, t)
+    if u.dim() != 3:
+        raise ValueError("u must be (batch, dim, L)")
+    if y is None:
+        y = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((u.shape[0], u.shape[1], A.shape[1]), dtype=torch.float32,
+                             pin_memory=True)
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last, host=True)
+    lib = _abi.load()
+    need = lib.ssm_scan_fwd_host_staging_size(ctypes.byref(a), int(slice_batch))
+    if need == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    if staging is None or staging.numel() * staging.element_size() < need:
+        staging = torch.empty(max(int(need), 1), dtype=torch.uint8, device="cuda")
+    _cuda("staging", staging)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    _abi.check(lib.ssm_scan_fwd_host(ctypes.byref(a), int(slice_batch), _ptr(staging),
+                                     staging.numel() * staging.element_size(),
+                                     ctypes.c_void_p(s.cuda_stream)),
+               "ssm_scan_fwd_host")
+    if synchronize:
+        s.synchronize()
     return y, h_last
 
 

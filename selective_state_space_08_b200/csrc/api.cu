@@ -419,6 +419,180 @@ cudaError_t noalloc_scratch(void** out) {
   return cudaSuccess;
 }
 
+// ---- host-resident scan: batch slices pipelined through device staging ------
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+struct HostPlan {
+  int64_t sb = 1, nslices = 0;
+  size_t es = 0, x_bytes = 0, bc_bytes = 0, h_bytes = 0;  // one full slice of u / B / h
+  size_t off_A = 0, off_D = 0, off_bias = 0, off_ws = 0, ws_bytes = 0, off_slot = 0;
+  // within a slot
+  size_t off_u = 0, off_dl = 0, off_z = 0, off_B = 0, off_C = 0, off_y = 0, off_h0 = 0, off_h = 0;
+  size_t slot_bytes = 0, total = 0;
+};
+
+ssm_status_t plan_host(const ssm_scan_args_t* a, int64_t sb, HostPlan* hp) {
+  if (a == nullptr || sb < 1) return SSM_ERR_INVALID_ARG;
+  const int64_t* strides[] = {a->u_stride, a->delta_stride, a->z_stride,
+                              a->y_stride, a->B_stride, a->C_stride};
+  for (const int64_t* st : strides)
+    if (st[0] != 0 || st[1] != 0) return SSM_ERR_UNSUPPORTED;
+  ScanPlan whole;
+  ssm_status_t st = plan_scan(a, &whole);  // sizes, flags and the host pointers
+  if (st != SSM_OK) return st;
+  hp->sb = sb < a->batch ? sb : (a->batch > 0 ? a->batch : 1);
+  hp->nslices = (a->batch + hp->sb - 1) / hp->sb;
+  // scratch of the scan of a full slice and of the last (possibly smaller) one
+  size_t ws = 0;
+  for (int64_t nb : {hp->sb, a->batch - (hp->nslices - 1) * hp->sb}) {
+    if (nb <= 0) continue;
+    ssm_scan_args_t sa = *a;
+    sa.batch = nb;
+    ScanPlan sp;
+    st = plan_scan(&sa, &sp, false);
+    if (st != SSM_OK) return st;
+    if (sp.ws_bytes > ws) ws = sp.ws_bytes;
+  }
+  const size_t es = elem_size(a->dtype);
+  const size_t D = static_cast<size_t>(a->dim), N = static_cast<size_t>(a->dstate);
+  const size_t L = static_cast<size_t>(a->seqlen), S = static_cast<size_t>(hp->sb);
+  hp->es = es;
+  hp->x_bytes = S * D * L * es;
+  hp->bc_bytes = S * N * L * es;
+  hp->h_bytes = S * D * N * sizeof(float);
+  size_t o = 0;
+  hp->off_A = o;    o += round256(D * N * sizeof(float));
+  hp->off_D = o;    o += a->D ? round256(D * sizeof(float)) : 0;
+  hp->off_bias = o; o += a->delta_bias ? round256(D * sizeof(float)) : 0;
+  hp->off_ws = o;   o += round256(ws);
+  hp->ws_bytes = ws;
+  hp->off_slot = o;
+  size_t q = 0;
+  hp->off_u = q;  q += round256(hp->x_bytes);
+  hp->off_dl = q; q += round256(hp->x_bytes);
+  hp->off_z = q;  q += a->z ? round256(hp->x_bytes) : 0;
+  hp->off_B = q;  q += round256(hp->bc_bytes);
+  hp->off_C = q;  q += round256(hp->bc_bytes);
+  hp->off_y = q;  q += round256(hp->x_bytes);
+  hp->off_h0 = q; q += a->h0 ? round256(hp->h_bytes) : 0;
+  hp->off_h = q;  q += a->h_last ? round256(hp->h_bytes) : 0;
+  hp->slot_bytes = q;
+  hp->total = o + 2 * q;
+  return SSM_OK;
+}
+
+// Two copy streams per device (host-to-device, device-to-host), created on
+// first use and kept for the life of the process.
+ssm_status_t copy_streams(cudaStream_t* in, cudaStream_t* out) {
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices][2] = {};
+  int dev = 0;
+  ssm_status_t st = cuda_status(cudaGetDevice(&dev), "scan_fwd_host: current device");
+  if (st != SSM_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return SSM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 2; ++i) {
+    if (streams[dev][i] == nullptr) {
+      st = cuda_status(cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking),
+                       "scan_fwd_host: copy stream");
+      if (st != SSM_OK) return st;
+    }
+  }
+  *in = streams[dev][0];
+  *out = streams[dev][1];
+  return SSM_OK;
+}
+
+// The queued work of one ssm_scan_fwd_host call (see include/ssmscan.h).
+ssm_status_t run_host(const ssm_scan_args_t* a, const HostPlan& hp, unsigned char* stg,
+                      cudaStream_t stream) {
+  cudaStream_t sin = nullptr, sout = nullptr;
+  ssm_status_t st = copy_streams(&sin, &sout);
+  if (st != SSM_OK) return st;
+  // start, then per slot: inputs in, scan done, outputs out
+  cudaEvent_t ev[7] = {};
+  for (cudaEvent_t& e : ev) {
+    st = cuda_status(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "scan_fwd_host: event");
+    if (st != SSM_OK) break;
+  }
+  cudaEvent_t ev_start = ev[0], *in_done = ev + 1, *comp_done = ev + 3, *out_done = ev + 5;
+  auto chk = [&](cudaError_t e, const char* what) {
+    if (st == SSM_OK) st = cuda_status(e, what);
+    return st == SSM_OK;
+  };
+  auto h2d = [&](void* dst, const void* src, size_t n) {
+    return n == 0 || chk(cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, sin),
+                         "scan_fwd_host: copy to device");
+  };
+  auto d2h = [&](void* dst, const void* src, size_t n) {
+    return n == 0 || chk(cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToHost, sout),
+                         "scan_fwd_host: copy to host");
+  };
+  const size_t D = static_cast<size_t>(a->dim), N = static_cast<size_t>(a->dstate);
+  const size_t L = static_cast<size_t>(a->seqlen), es = hp.es;
+  if (st == SSM_OK && chk(cudaEventRecord(ev_start, stream), "scan_fwd_host: record") &&
+      chk(cudaStreamWaitEvent(sin, ev_start, 0), "scan_fwd_host: wait") &&
+      chk(cudaStreamWaitEvent(sout, ev_start, 0), "scan_fwd_host: wait") &&
+      h2d(stg + hp.off_A, a->A, D * N * sizeof(float)) &&
+      (a->D == nullptr || h2d(stg + hp.off_D, a->D, D * sizeof(float))) &&
+      (a->delta_bias == nullptr || h2d(stg + hp.off_bias, a->delta_bias, D * sizeof(float)))) {
+    for (int64_t s = 0; s < hp.nslices && st == SSM_OK; ++s) {
+      const int k = static_cast<int>(s & 1);
+      unsigned char* slot = stg + hp.off_slot + k * hp.slot_bytes;
+      const int64_t b0 = s * hp.sb;
+      const int64_t nb = a->batch - b0 < hp.sb ? a->batch - b0 : hp.sb;
+      const size_t xo = static_cast<size_t>(b0) * D * L * es, xn = static_cast<size_t>(nb) * D * L * es;
+      const size_t bo = static_cast<size_t>(b0) * N * L * es, bn = static_cast<size_t>(nb) * N * L * es;
+      const size_t ho = static_cast<size_t>(b0) * D * N * sizeof(float);
+      const size_t hn = static_cast<size_t>(nb) * D * N * sizeof(float);
+      auto in = [](const void* base, size_t off) {
+        return static_cast<const unsigned char*>(base) + off;
+      };
+      // slot k's inputs were last read by the scan of slice s - 2
+      if (s >= 2 && !chk(cudaStreamWaitEvent(sin, comp_done[k], 0), "scan_fwd_host: wait")) break;
+      if (!(h2d(slot + hp.off_u, in(a->u, xo), xn) && h2d(slot + hp.off_dl, in(a->delta, xo), xn) &&
+            (a->z == nullptr || h2d(slot + hp.off_z, in(a->z, xo), xn)) &&
+            h2d(slot + hp.off_B, in(a->B, bo), bn) && h2d(slot + hp.off_C, in(a->C, bo), bn) &&
+            (a->h0 == nullptr || h2d(slot + hp.off_h0, in(a->h0, ho), hn)) &&
+            chk(cudaEventRecord(in_done[k], sin), "scan_fwd_host: record") &&
+            chk(cudaStreamWaitEvent(stream, in_done[k], 0), "scan_fwd_host: wait")))
+        break;
+      // slot k's outputs of slice s - 2 must have left before the scan rewrites them
+      if (s >= 2 && !chk(cudaStreamWaitEvent(stream, out_done[k], 0), "scan_fwd_host: wait")) break;
+      ssm_scan_args_t sa = *a;
+      sa.batch = nb;
+      sa.u = slot + hp.off_u;
+      sa.delta = slot + hp.off_dl;
+      sa.z = a->z ? slot + hp.off_z : nullptr;
+      sa.B = slot + hp.off_B;
+      sa.C = slot + hp.off_C;
+      sa.y = slot + hp.off_y;
+      sa.h0 = a->h0 ? reinterpret_cast<const float*>(slot + hp.off_h0) : nullptr;
+      sa.h_last = a->h_last ? reinterpret_cast<float*>(slot + hp.off_h) : nullptr;
+      sa.A = reinterpret_cast<const float*>(stg + hp.off_A);
+      sa.D = a->D ? reinterpret_cast<const float*>(stg + hp.off_D) : nullptr;
+      sa.delta_bias = a->delta_bias ? reinterpret_cast<const float*>(stg + hp.off_bias) : nullptr;
+      st = ssm_scan_fwd(&sa, hp.ws_bytes ? stg + hp.off_ws : nullptr, hp.ws_bytes,
+                        reinterpret_cast<ssm_stream_t>(stream));
+      if (st != SSM_OK) break;
+      if (!(chk(cudaEventRecord(comp_done[k], stream), "scan_fwd_host: record") &&
+            chk(cudaStreamWaitEvent(sout, comp_done[k], 0), "scan_fwd_host: wait") &&
+            d2h(static_cast<unsigned char*>(a->y) + xo, slot + hp.off_y, xn) &&
+            (a->h_last == nullptr ||
+             d2h(reinterpret_cast<unsigned char*>(a->h_last) + ho, slot + hp.off_h, hn)) &&
+            chk(cudaEventRecord(out_done[k], sout), "scan_fwd_host: record")))
+        break;
+    }
+    // the caller's stream finishes when every copy back has landed
+    for (int k = 0; k < 2 && k < hp.nslices && st == SSM_OK; ++k)
+      chk(cudaStreamWaitEvent(stream, out_done[k], 0), "scan_fwd_host: wait");
+  }
+  for (cudaEvent_t e : ev)
+    if (e != nullptr) cudaEventDestroy(e);  // released once the queued work has used them
+  return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -452,6 +626,24 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t w
     return plan.vec ? run_fwd<__nv_bfloat16, true>(p, stream)
                     : run_fwd<__nv_bfloat16, false>(p, stream);
   return plan.vec ? run_fwd<float, true>(p, stream) : run_fwd<float, false>(p, stream);
+}
+
+size_t ssm_scan_fwd_host_staging_size(const ssm_scan_args_t* args, int64_t slice_batch) {
+  HostPlan hp;
+  if (plan_host(args, slice_batch, &hp) != SSM_OK) return static_cast<size_t>(-1);
+  return hp.total;
+}
+
+ssm_status_t ssm_scan_fwd_host(const ssm_scan_args_t* args, int64_t slice_batch, void* staging,
+                               size_t staging_bytes, ssm_stream_t stream) {
+  HostPlan hp;
+  ssm_status_t st = plan_host(args, slice_batch, &hp);
+  if (st != SSM_OK) return st;
+  if (args->batch == 0 || args->dim == 0) return SSM_OK;
+  if (staging == nullptr || staging_bytes < hp.total) return SSM_ERR_WORKSPACE;
+  if (!aligned(staging, 256)) return SSM_ERR_ALIGNMENT;
+  return run_host(args, hp, static_cast<unsigned char*>(staging),
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 ssm_status_t ssm_scan_fwd_noalloc(const ssm_scan_args_t* args, ssm_stream_t stream) {

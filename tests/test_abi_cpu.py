@@ -90,6 +90,27 @@ def test_empty_problems_are_no_ops(lib):
     assert lib.ssm_scan_fwd(ctypes.byref(a), None, 0, None) == 0
 
 
+def test_host_scan_staging_and_host_side_errors(lib):
+    """ssm_scan_fwd_host: staging grows with the slice up to the whole batch;
+    bad slices and strided layouts are refused; missing or short staging is
+    reported before anything touches a GPU."""
+    a = _args(batch=5, dim=64, seqlen=300)
+    size = [lib.ssm_scan_fwd_host_staging_size(ctypes.byref(a), sb) for sb in (1, 2, 5, 9)]
+    assert 0 < size[0] < size[1] < size[2] == size[3]
+    bad = ctypes.c_size_t(-1).value
+    assert lib.ssm_scan_fwd_host_staging_size(ctypes.byref(a), 0) == bad
+    assert lib.ssm_scan_fwd_host_staging_size(None, 1) == bad
+    s = _args(batch=5, dim=64, seqlen=300)
+    s.u_stride[1] = 512
+    assert lib.ssm_scan_fwd_host_staging_size(ctypes.byref(s), 1) == bad
+    assert lib.ssm_scan_fwd_host(ctypes.byref(s), 1, 0x10000, 1 << 30, None) == 2
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), 0, 0x10000, 1 << 30, None) == 1
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), 2, None, 0, None) == 5
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), 2, 0x10000, size[1] - 1, None) == 5
+    assert lib.ssm_scan_fwd_host(ctypes.byref(a), 2, 0x10010, size[1], None) == 3
+    assert lib.ssm_scan_fwd_host(ctypes.byref(_args(batch=0)), 1, None, 0, None) == 0
+
+
 def test_step_rejects_bad_arguments(lib):
     s = _abi.StepArgs()
     s.batch, s.dim, s.dstate, s.dtype = 2, 3, 16, 0
