@@ -314,7 +314,7 @@ def time_steps(step, steps, warmup, flush, world, device, sampler_index=None):
     return total, per, sampler.record()
 
 
-def e2e_measure(case, steps, warmup, slice_batch=1):
+def e2e_measure(case, steps, warmup, slice_batch=2):
     """The same metric through the C ABI from page-locked host buffers
     (ssm_scan_fwd_host): per step the host->device copies of every input, the
     scan and the device->host copies of y and h_last, all inside the timed
