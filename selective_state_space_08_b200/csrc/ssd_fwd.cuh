@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(256) ssd_pass_kernel(const SsdParams p) {
   if (idx >= p.batch * p.nheads * per) return;
   const int64_t bh = idx / per, e = idx % per;  // e = p * N + n
   float s = p.h0 ? p.h0[idx] : 0.f;             // h0 is (b, h, p, n): same order
-  constexpr int kAhead = 4;                      // loads issued ahead of the dependent chain
+  constexpr int kAhead = 8;                      // loads issued ahead of the dependent chain
   int64_t c = 0;
   for (; c + kAhead <= p.nchunks; c += kAhead) {
     float sl[kAhead], ce[kAhead];

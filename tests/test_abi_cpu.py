@@ -111,6 +111,30 @@ def test_host_scan_staging_and_host_side_errors(lib):
     assert lib.ssm_scan_fwd_host(ctypes.byref(_args(batch=0)), 1, None, 0, None) == 0
 
 
+def _ssd_args(**kw):
+    a = _abi.SsdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.chunk = 2, 1000, 8, 64, 128, 256
+    a.dtype = _abi.SSM_BF16
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_chunked_scan_sizes_and_limits(lib):
+    """The chunked scan's workspace query accepts the implemented sizes and
+    refuses the others, including sizes past the 32-bit TMA coordinates."""
+    bad = ctypes.c_size_t(-1).value
+    ok = lib.ssm_scan_fwd_chunked_workspace_size(ctypes.byref(_ssd_args()))
+    assert 0 < ok < (1 << 30)
+    assert lib.ssm_scan_fwd_chunked_workspace_size(ctypes.byref(_ssd_args(chunk=128))) > ok
+    for kw in (dict(headdim=32), dict(dstate=64), dict(chunk=64), dict(dtype=_abi.SSM_F32),
+               dict(batch=-1), dict(seqlen=(1 << 31)),
+               dict(batch=4096, nheads=4096, seqlen=1024)):  # 4096*4096*4 chunks * 64 rows
+        assert lib.ssm_scan_fwd_chunked_workspace_size(ctypes.byref(_ssd_args(**kw))) == bad, kw
+    assert lib.ssm_scan_fwd_chunked(ctypes.byref(_ssd_args()), None, 0, None) == 1  # null pointers
+    assert lib.ssm_scan_fwd_chunked(ctypes.byref(_ssd_args(batch=0)), None, 0, None) == 0
+
+
 def test_step_rejects_bad_arguments(lib):
     s = _abi.StepArgs()
     s.batch, s.dim, s.dstate, s.dtype = 2, 3, 16, 0
