@@ -64,6 +64,8 @@ def _bind(lib):
     lib.oracle_ssd_fwd.argtypes = [_i64] * 5 + [_dp] * 8 + [ctypes.c_int, _dp, _dp, _dp,
                                                             ctypes.c_int]
     lib.oracle_ssd_fwd.restype = ctypes.c_int
+    lib.oracle_conv_silu.argtypes = [_i64] * 4 + [_dp] * 5 + [ctypes.c_int]
+    lib.oracle_conv_silu.restype = ctypes.c_int
     return lib
 
 
@@ -109,6 +111,37 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     if rc != 0:
         raise RuntimeError(f"oracle_scan_fwd failed ({rc})")
     return y, h_last
+
+
+def conv_silu(x, w, bias=None, x_prev=None, nthreads=None, lib=None):
+    """Causal depthwise convolution over time, then SiLU (the input stage of
+    the scan).  x: (batch, dim, L); w: (dim, width); bias: (dim);
+    x_prev: (batch, dim, width - 1), the inputs just before step 0 in time
+    order (zeros when None).  Returns u (batch, dim, L) in float64."""
+    x = _f64(x)
+    batch, dim, L = x.shape
+    w = _f64(w)
+    if w.ndim != 2 or w.shape[0] != dim or w.shape[1] < 1:
+        raise ValueError(f"w must be (dim, width), got {w.shape}")
+    K = w.shape[1]
+    bias = _f64(bias, (dim,))
+    x_prev = _f64(x_prev, (batch, dim, K - 1))
+    u = np.zeros((batch, dim, L), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_conv_silu(batch, dim, L, K, _p(x), _p(w), _p(bias), _p(x_prev), _p(u),
+                              int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle_conv_silu failed ({rc})")
+    return u
+
+
+def scan_fwd_conv(x, conv_w, conv_bias, x_prev, delta, A, B, C, D=None, z=None,
+                  delta_bias=None, delta_softplus=True, h0=None, nthreads=None, lib=None):
+    """The scan fed by the convolution stage: u = conv_silu(x, ...), then
+    scan_fwd(u, ...).  Returns (y, h_last) in float64."""
+    u = conv_silu(x, conv_w, conv_bias, x_prev, nthreads=nthreads, lib=lib)
+    return scan_fwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, nthreads=nthreads,
+                    lib=lib)
 
 
 def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,

@@ -234,4 +234,64 @@ int oracle_ssd_fwd(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdi
   return 0;
 }
 
-int oracle_abi_version(void) { return 1; }
+/* ------------------------------------------------------------------ */
+/* Causal depthwise convolution over time followed by SiLU, in front of the
+ * scan.  [P2] section 3 (block flow: a local convolution captures
+ * short-range patterns before the selective SSM; SiLU is the block's
+ * activation; kernel size 4 among the block's hyperparameters).  Readings
+ * (the page gives no formula): causal, one filter of `width` taps per
+ * channel, the last tap on the current step, then the channel's bias:
+ *   u[b,d,t] = silu(bias_d + sum_{k<width} w[d,k] x[b,d,t-(width-1)+k]);
+ * inputs at negative times come from x_prev (batch, dim, width-1), whose
+ * entry j is the input at time j-(width-1), or are zero without it.
+ * x, u : (batch, dim, seqlen)   w : (dim, width)   bias : (dim) */
+typedef struct {
+  int64_t dim, seqlen, width;
+  const double *x, *w, *bias, *x_prev;
+  double* u;
+  int64_t row_begin, row_end;
+} conv_job;
+
+static void* conv_rows(void* arg) {
+  const conv_job* j = (const conv_job*)arg;
+  const int64_t L = j->seqlen, K = j->width;
+  for (int64_t row = j->row_begin; row < j->row_end; ++row) {
+    const int64_t d = row % j->dim;
+    for (int64_t t = 0; t < L; ++t) {
+      double acc = j->bias ? j->bias[d] : 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        const int64_t tt = t - (K - 1) + k; /* time of the input under tap k */
+        double xv = 0.0;
+        if (tt >= 0)
+          xv = j->x[row * L + tt];
+        else if (j->x_prev)
+          xv = j->x_prev[row * (K - 1) + tt + (K - 1)];
+        acc += j->w[d * K + k] * xv;
+      }
+      j->u[row * L + t] = silu_d(acc);
+    }
+  }
+  return NULL;
+}
+
+static void conv_set_range(void* p, int64_t a, int64_t b) {
+  ((conv_job*)p)->row_begin = a;
+  ((conv_job*)p)->row_end = b;
+}
+
+int oracle_conv_silu(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, const double* x,
+                     const double* w, const double* bias, const double* x_prev, double* u,
+                     int nthreads) {
+  if (batch < 0 || dim < 0 || seqlen < 0 || width < 1) return -1;
+  const int64_t rows = batch * dim;
+  if (rows == 0 || seqlen == 0) return 0;
+  if (nthreads < 1) nthreads = 1;
+  conv_job* jobs = (conv_job*)calloc((size_t)nthreads, sizeof(conv_job));
+  for (int i = 0; i < nthreads; ++i)
+    jobs[i] = (conv_job){dim, seqlen, width, x, w, bias, x_prev, u, 0, 0};
+  run_parallel(conv_rows, jobs, sizeof(conv_job), rows, nthreads, conv_set_range);
+  free(jobs);
+  return 0;
+}
+
+int oracle_abi_version(void) { return 2; }

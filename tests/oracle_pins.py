@@ -405,8 +405,87 @@ def pin_ssd_chunked(lib):
         _close(h_last, hc, what=f"SSD chunk {q} h_L")
 
 
+# ---- the convolution stage in front of the scan -------------------------------
+# Page "从硬件感知到算法革命" (tencentcloud) §3: a local convolution over time
+# (kernel size 4) feeds the selective SSM; SiLU is the block's activation.
+
+
+def _rand_conv(rng, batch=2, dim=3, L=30, K=4, prev=True):
+    x = rng.standard_normal((batch, dim, L))
+    w = rng.standard_normal((dim, K)) * 0.7
+    b = rng.standard_normal(dim) * 0.3
+    xp = rng.standard_normal((batch, dim, K - 1)) if prev and K > 1 else None
+    return x, w, b, xp
+
+
+def _conv_numpy(x, w, b, xp):
+    """The causal depthwise convolution by np.convolve: the channel's inputs
+    with the preceding window prepended, convolved with the taps reversed
+    (np.convolve flips its kernel), the causal outputs kept; then SiLU."""
+    batch, dim, L = x.shape
+    K = w.shape[1]
+    out = np.empty_like(x)
+    for bb in range(batch):
+        for d in range(dim):
+            prev = xp[bb, d] if xp is not None else np.zeros(K - 1)
+            xe = np.concatenate([prev, x[bb, d]])
+            pre = np.convolve(xe, w[d, ::-1])[K - 1:K - 1 + L] + (b[d] if b is not None else 0.0)
+            out[bb, d] = _silu(pre)
+    return out
+
+
+def pin_conv_numpy(lib):
+    """C1: the convolution stage equals np.convolve's causal outputs plus the
+    bias, through SiLU, for widths 1..4, with and without the preceding
+    window and the bias."""
+    rng = np.random.default_rng(31)
+    for K in (1, 2, 3, 4):
+        for prev in (True, False):
+            x, w, b, xp = _rand_conv(rng, K=K, prev=prev)
+            for bias in (b, None):
+                got = oracle.conv_silu(x, w, bias, xp, lib=lib)
+                _close(got, _conv_numpy(x, w, bias, xp), what=f"conv K={K} prev={prev}")
+
+
+def pin_conv_one_tap(lib):
+    """C2: one tap of weight 1 and no bias leave u = silu(x) = x expit(x)."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((2, 3, 17)) * 3
+    got = oracle.conv_silu(x, np.ones((3, 1)), None, None, lib=lib)
+    _close(got, x * expit(x), what="one-tap conv")
+
+
+def pin_conv_split_resume(lib):
+    """C3: convolving [0, m) and then [m, L) with the last width-1 inputs
+    before m as the preceding window gives the one-pass result."""
+    rng = np.random.default_rng(33)
+    x, w, b, xp = _rand_conv(rng, L=40, K=4)
+    whole = oracle.conv_silu(x, w, b, xp, lib=lib)
+    m = 13
+    first = oracle.conv_silu(x[..., :m], w, b, xp, lib=lib)
+    second = oracle.conv_silu(x[..., m:], w, b, x[..., m - 3:m], lib=lib)
+    _close(np.concatenate([first, second], axis=-1), whole, what="conv split/resume")
+
+
+def pin_conv_feeds_scan(lib):
+    """C4: the convolution stage runs before the scan and its output is the u
+    of both the input term and the skip term: scan_fwd_conv equals the scan
+    fed with the np.convolve reference of the stage."""
+    rng = np.random.default_rng(34)
+    inp = _rand_scan(rng, L=26)
+    x, w, b, xp = _rand_conv(rng, batch=2, dim=3, L=26, K=4)
+    y, h = oracle.scan_fwd_conv(x, w, b, xp, inp["delta"], inp["A"], inp["B"], inp["C"],
+                                inp["D"], inp["z"], inp["delta_bias"], True, inp["h0"], lib=lib)
+    u = _conv_numpy(x, w, b, xp)
+    yr, hr = oracle.scan_fwd(u, inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"],
+                             inp["delta_bias"], True, inp["h0"], lib=lib)
+    _close(y, yr, what="conv feeding the scan: y")
+    _close(h, hr, what="conv feeding the scan: h_L")
+
+
 MAMBA1_PINS = [pin_closed_form, pin_augmented_matrix, pin_blelloch_order, pin_lti_convolution,
                pin_split_resume, pin_prefix_sum_case, pin_memoryless_case, pin_gate_and_skip,
                pin_softplus_and_bias, pin_decode_steps]
 SSD_PINS = [pin_ssd_is_mamba1, pin_ssd_quadratic, pin_ssd_chunked]
-ALL_PINS = MAMBA1_PINS + SSD_PINS
+CONV_PINS = [pin_conv_numpy, pin_conv_one_tap, pin_conv_split_resume, pin_conv_feeds_scan]
+ALL_PINS = MAMBA1_PINS + SSD_PINS + CONV_PINS

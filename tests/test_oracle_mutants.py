@@ -12,7 +12,7 @@ import subprocess
 import pytest
 
 import oracle
-from oracle_pins import ALL_PINS, MAMBA1_PINS, SSD_PINS
+from oracle_pins import ALL_PINS, CONV_PINS, MAMBA1_PINS, SSD_PINS
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
 
@@ -44,6 +44,13 @@ MUTANTS = [
     ("ssd_readout_uses_B", "acc += Ct[n] * S[p * N + n];", "acc += Bt[n] * S[p * N + n];", SSD_PINS),
     ("ssd_drop_skip", "(j->D ? j->D[hd] * xv : 0.0)", "0.0", SSD_PINS),
     ("ssd_ignore_h0", "S[i] = j->h0 ? j->h0[row * P * N + i] : 0.0;", "S[i] = 0.0;", SSD_PINS),
+    ("conv_taps_reversed", "acc += j->w[d * K + k] * xv;", "acc += j->w[d * K + (K - 1 - k)] * xv;",
+     CONV_PINS),
+    ("conv_no_bias", "double acc = j->bias ? j->bias[d] : 0.0;", "double acc = 0.0;", CONV_PINS),
+    ("conv_no_silu", "j->u[row * L + t] = silu_d(acc);", "j->u[row * L + t] = acc;", CONV_PINS),
+    ("conv_ignores_window", "else if (j->x_prev)", "else if (0)", CONV_PINS),
+    ("conv_time_shift", "const int64_t tt = t - (K - 1) + k;", "const int64_t tt = t - K + k;",
+     CONV_PINS),
 ]
 
 
