@@ -444,6 +444,27 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
                     "launches_per_call": case.launches}
         del case
         torch.cuda.empty_cache()
+    # the scan with the convolution stage fused in front (width 4), 130M-layer shape
+    case = ScanCase(WORKLOAD)
+    conv = synth.make_conv_params(case.cfg["dim"], 4, seed=1)
+    cw = torch.from_numpy(conv["weight"]).cuda()
+    cb = torch.from_numpy(conv["bias"]).cuda()
+    t = case.t
+    cstep = lambda: api.scan_fwd_conv(t["u"], cw, cb, None, t["delta"], t["A"], t["B"], t["C"],
+                                      t["D"], t["z"], t["delta_bias"], True, None, y=case.y,
+                                      h_last=case.h, workspace=case.ws)
+    total, per, _ = time_steps(cstep, steps, warmup, flush, 1, None)
+    sec = total / steps
+    cbytes = case.bytes + cw.numel() * 4 + cb.numel() * 4
+    out["mamba130m_layer_conv"] = {
+        "config": describe(case.cfg, True) + ", conv width 4 fused in front",
+        "us_per_call": round(sec * 1e6, 2), "GB_per_s": round(cbytes / sec / 1e9, 1),
+        "hbm_frac": round(cbytes / sec / 1e9 / hbm_peak, 4),
+        "elems_per_s": round(case.elems / sec, 1),
+        "alu_frac": round(case.elems / sec / alu_peak_elems(case.cfg["dstate"], True), 4),
+        "launches_per_call": case.launches}
+    del case, cstep
+    torch.cuda.empty_cache()
     # Mamba-2 chunked scan (tensor cores)
     cfg, sstep, keep = ssd_case()
     total, per, _ = time_steps(sstep, steps, warmup, flush, 1, None)

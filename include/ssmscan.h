@@ -122,6 +122,31 @@ size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args);
 ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t workspace_bytes,
                           ssm_stream_t stream);
 
+/* The selective scan with the block's convolution stage in front, fused
+ * into the same kernel so that the stage's input is read from HBM once.
+ * Page "从硬件感知到算法革命：Mamba如何重塑序列建模的计算效率", section 3 (a
+ * local convolution over time before the selective SSM, kernel size 4;
+ * SiLU as the block's activation).  `args` is that of ssm_scan_fwd except
+ * that args->u holds the stage's input x; the scan then runs on
+ *   u[b,d,t] = silu(bias_d + sum_{k<width} weight[d,k] x[b,d,t-(width-1)+k]),
+ * which also feeds the skip term D*u.  Inputs before step 0 come from x_prev
+ * (entry j is the input at step j-(width-1)), or are zero when it is NULL.
+ *   width  : 1..4 taps (others: SSM_ERR_UNSUPPORTED);
+ *   weight : (dim, width) fp32, required;  bias : (dim) fp32 or NULL;
+ *   x_prev : (batch, dim, width-1) fp32, contiguous, or NULL.
+ * Workspace: as for ssm_scan_fwd (ssm_scan_fwd_workspace_size of `args`).
+ * Split-and-resume: pass the last width-1 inputs of the first part as x_prev
+ * of the second (together with h0 = h_last). */
+typedef struct {
+  int64_t width;
+  const float* weight;
+  const float* bias;
+  const float* x_prev;
+} ssm_conv_args_t;
+
+ssm_status_t ssm_scan_fwd_conv(const ssm_scan_args_t* args, const ssm_conv_args_t* conv,
+                               void* workspace, size_t workspace_bytes, ssm_stream_t stream);
+
 /* Bytes of the library's static device scratch used by ssm_scan_fwd_noalloc. */
 #define SSM_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 

@@ -33,6 +33,10 @@ class ScanArgs(ctypes.Structure):
                 ("y_stride", _i64 * 2), ("B_stride", _i64 * 2), ("C_stride", _i64 * 2)]
 
 
+class ConvArgs(ctypes.Structure):
+    _fields_ = [("width", _i64), ("weight", _fp), ("bias", _fp), ("x_prev", _fp)]
+
+
 class StepArgs(ctypes.Structure):
     _fields_ = [("batch", _i64), ("dim", _i64), ("dstate", _i64), ("dtype", ctypes.c_int),
                 ("u", _vp), ("delta", _vp), ("z", _vp), ("B", _vp), ("C", _vp),
@@ -73,6 +77,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_scan_fwd_workspace_size.restype = ctypes.c_size_t
     lib.ssm_scan_fwd.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.c_size_t, _vp]
     lib.ssm_scan_fwd.restype = ctypes.c_int
+    lib.ssm_scan_fwd_conv.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ConvArgs), _vp,
+                                      ctypes.c_size_t, _vp]
+    lib.ssm_scan_fwd_conv.restype = ctypes.c_int
     lib.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _vp]
     lib.ssm_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_scan_fwd_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), _i64]

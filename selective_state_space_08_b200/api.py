@@ -133,6 +133,50 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     return y, h_last
 
 
+def scan_fwd_conv(x, conv_weight, conv_bias, x_prev, delta, A, B, C, D=None, z=None,
+                  delta_bias=None, delta_softplus=True, h0=None, *, y=None, h_last=None,
+                  return_last_state=True, workspace=None, stream=None):
+    """The scan with the convolution stage in front, in one kernel: u =
+    silu(conv_bias + causal depthwise conv(x)) feeds the scan and the skip
+    term.  x: (batch, dim, L) like ``scan_fwd``'s u; conv_weight: (dim,
+    width) float32, width 1..4; conv_bias: (dim,) float32 or None; x_prev:
+    (batch, dim, width - 1) float32 or None (inputs before step 0).
+    Returns (y, h_last)."""
+    for name, t in (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+        _cuda(name, t)
+    if x.dim() != 3:
+        raise ValueError("x must be (batch, dim, L)")
+    batch, dim, _ = x.shape
+    _cuda("conv_weight", conv_weight, torch.float32, 2)
+    width = conv_weight.shape[1]
+    if tuple(conv_weight.shape) != (dim, width) or not conv_weight.is_contiguous():
+        raise ValueError("conv_weight must be contiguous float32 of shape (dim, width)")
+    for name, t, shape in (("conv_bias", conv_bias, (dim,)),
+                           ("x_prev", x_prev, (batch, dim, width - 1))):
+        if t is not None:
+            _cuda(name, t, torch.float32)
+            if tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be contiguous float32 of shape {shape}")
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((batch, dim, A.shape[1]), dtype=torch.float32, device=x.device)
+    a = _scan_args(x, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last)
+    c = _abi.ConvArgs()
+    c.width, c.weight, c.bias, c.x_prev = width, _ptr(conv_weight), _ptr(conv_bias), _ptr(x_prev)
+    lib = _abi.load()
+    need = lib.ssm_scan_fwd_workspace_size(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(int(need), dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _abi.check(lib.ssm_scan_fwd_conv(ctypes.byref(a), ctypes.byref(c), _ptr(workspace), ws_bytes,
+                                     _stream(stream)), "ssm_scan_fwd_conv")
+    return y, h_last
+
+
 def scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                      h0=None, *, y, h_last=None, stream=None):
     """``scan_fwd`` for callers that cannot allocate device memory: ``y`` (and

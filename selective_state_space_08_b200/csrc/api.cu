@@ -171,10 +171,10 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* out, bool check_ptrs 
   return SSM_OK;
 }
 
-template <typename T, int MODE, bool HAS_Z, bool VEC>
+template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV>
 ssm_status_t launch_fwd(const ScanParams& p, cudaStream_t stream) {
-  auto kernel = fwd::scan_fwd_kernel<T, MODE, HAS_Z, VEC>;
-  const size_t smem = sizeof(fwd::Smem<T>);
+  auto kernel = fwd::scan_fwd_kernel<T, MODE, HAS_Z, VEC, CONV>;
+  const size_t smem = sizeof(fwd::Smem<T, CONV>);
   ssm_status_t st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem),
                                 "scan_fwd: shared-memory opt-in");
   if (st != SSM_OK) return st;
@@ -186,11 +186,11 @@ ssm_status_t launch_fwd(const ScanParams& p, cudaStream_t stream) {
                                                            : "scan_fwd: scan pass launch");
 }
 
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool CONV>
 ssm_status_t run_fwd(const ScanParams& p, cudaStream_t stream) {
   ssm_status_t st = SSM_OK;
   if (p.nseg > 1) {
-    st = launch_fwd<T, fwd::kAgg, false, VEC>(p, stream);
+    st = launch_fwd<T, fwd::kAgg, false, VEC, CONV>(p, stream);
     if (st != SSM_OK) return st;
     const int64_t total = p.batch * p.dim * fwd::kMaxN;
     const int threads = 256;
@@ -199,8 +199,8 @@ ssm_status_t run_fwd(const ScanParams& p, cudaStream_t stream) {
     st = cuda_status(cudaGetLastError(), "scan_fwd: carry launch");
     if (st != SSM_OK) return st;
   }
-  return p.z != nullptr ? launch_fwd<T, fwd::kFull, true, VEC>(p, stream)
-                        : launch_fwd<T, fwd::kFull, false, VEC>(p, stream);
+  return p.z != nullptr ? launch_fwd<T, fwd::kFull, true, VEC, CONV>(p, stream)
+                        : launch_fwd<T, fwd::kFull, false, VEC, CONV>(p, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -593,22 +593,26 @@ ssm_status_t run_host(const ssm_scan_args_t* a, const HostPlan& hp, unsigned cha
   return st;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args) {
-  ScanPlan plan;
-  if (plan_scan(args, &plan, false) != SSM_OK) return static_cast<size_t>(-1);
-  return plan.ws_bytes;
-}
-
-ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t workspace_bytes,
-                          ssm_stream_t stream_) {
+// ssm_scan_fwd, with the convolution stage in front when `conv` is given.
+ssm_status_t scan_fwd_impl(const ssm_scan_args_t* args, const ssm_conv_args_t* conv,
+                           void* workspace, size_t workspace_bytes, ssm_stream_t stream_) {
   ScanPlan plan;
   ssm_status_t st = plan_scan(args, &plan);
   if (st != SSM_OK) return st;
   ScanParams& p = plan.p;
+  p.conv_width = 0;
+  p.conv_w = p.conv_b = p.conv_prev = nullptr;
+  if (conv != nullptr) {
+    if (conv->width < 1 || conv->width > fwd::kMaxConv) return SSM_ERR_UNSUPPORTED;
+    if (p.batch > 0 && p.dim > 0 && conv->weight == nullptr) return SSM_ERR_INVALID_ARG;
+    const void* f32s[] = {conv->weight, conv->bias, conv->x_prev};
+    for (const void* t : f32s)
+      if (t != nullptr && !aligned(t, 4)) return SSM_ERR_ALIGNMENT;
+    p.conv_width = static_cast<int>(conv->width);
+    p.conv_w = conv->weight;
+    p.conv_b = conv->bias;
+    p.conv_prev = conv->width > 1 ? conv->x_prev : nullptr;
+  }
   if (p.batch == 0 || p.dim == 0) return SSM_OK;
   if (plan.ws_bytes > 0) {
     if (workspace == nullptr || workspace_bytes < plan.ws_bytes) return SSM_ERR_WORKSPACE;
@@ -622,10 +626,38 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t w
     p.carry_dt = nullptr;
   }
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  if (args->dtype == SSM_BF16)
-    return plan.vec ? run_fwd<__nv_bfloat16, true>(p, stream)
-                    : run_fwd<__nv_bfloat16, false>(p, stream);
-  return plan.vec ? run_fwd<float, true>(p, stream) : run_fwd<float, false>(p, stream);
+  const bool bf16 = args->dtype == SSM_BF16;
+  if (conv != nullptr) {
+    if (bf16)
+      return plan.vec ? run_fwd<__nv_bfloat16, true, true>(p, stream)
+                      : run_fwd<__nv_bfloat16, false, true>(p, stream);
+    return plan.vec ? run_fwd<float, true, true>(p, stream) : run_fwd<float, false, true>(p, stream);
+  }
+  if (bf16)
+    return plan.vec ? run_fwd<__nv_bfloat16, true, false>(p, stream)
+                    : run_fwd<__nv_bfloat16, false, false>(p, stream);
+  return plan.vec ? run_fwd<float, true, false>(p, stream) : run_fwd<float, false, false>(p, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args) {
+  ScanPlan plan;
+  if (plan_scan(args, &plan, false) != SSM_OK) return static_cast<size_t>(-1);
+  return plan.ws_bytes;
+}
+
+ssm_status_t ssm_scan_fwd(const ssm_scan_args_t* args, void* workspace, size_t workspace_bytes,
+                          ssm_stream_t stream_) {
+  return scan_fwd_impl(args, nullptr, workspace, workspace_bytes, stream_);
+}
+
+ssm_status_t ssm_scan_fwd_conv(const ssm_scan_args_t* args, const ssm_conv_args_t* conv,
+                               void* workspace, size_t workspace_bytes, ssm_stream_t stream) {
+  if (conv == nullptr) return SSM_ERR_INVALID_ARG;
+  return scan_fwd_impl(args, conv, workspace, workspace_bytes, stream);
 }
 
 size_t ssm_scan_fwd_host_staging_size(const ssm_scan_args_t* args, int64_t slice_batch) {

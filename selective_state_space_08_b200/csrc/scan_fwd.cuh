@@ -64,6 +64,12 @@ struct ScanParams {
   int64_t nseg, seg_len;
   float* carry_h;   // ((nseg - 1) * batch * dim) x 16
   float* carry_dt;  // (nseg - 1) * batch * dim
+  // Convolution stage in front of the scan (page "从硬件感知到算法革命",
+  // section 3): u = silu(bias + causal depthwise conv(x)), x passed as `u`.
+  int conv_width;           // 1..4 taps; 0: no convolution stage
+  const float* conv_w;      // (dim, conv_width)
+  const float* conv_b;      // (dim) or null
+  const float* conv_prev;   // (batch, dim, conv_width - 1) inputs before step 0, or null
 };
 
 namespace fwd {
@@ -84,7 +90,7 @@ constexpr float kMaxDecayArg = 126.0f;
 // one quarter-warp then land in 8 distinct 4-bank groups.
 constexpr int kBCRow = kMaxN + 4;
 
-template <typename T>
+template <typename T, bool CONV = false>
 struct Smem {
   static constexpr int kEPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
   // A raw row holds a tile plus a 16-byte pad, so consecutive rows start 4
@@ -99,7 +105,12 @@ struct Smem {
   float du[kCH][kTL + 4];    // dt' * u
   float Bf[kTL][kBCRow];     // fp32 B, [step][state]
   float Cf[kTL][kBCRow];
+  // convolution output u (fp32) for the epilogue's skip term; rows of 72
+  // floats put the epilogue's 8-byte reads on distinct banks
+  float uc[CONV ? kCH : 1][kTL + 8];
 };
+
+constexpr int kMaxConv = 4;  // taps of the convolution stage
 
 // softplus for a pair (see softplus_f in common.cuh for the three ranges; the
 // series threshold here is e^s < 1/16, with 6 terms).
@@ -266,10 +277,10 @@ __device__ __forceinline__ void sub_decays(const float* dtp_row, float2 A01, flo
   }
 }
 
-template <typename T, int MODE, bool HAS_Z, bool VEC>
+template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV = false>
 __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  Smem<T>& sm = *reinterpret_cast<Smem<T>*>(smem_raw);
+  Smem<T, CONV>& sm = *reinterpret_cast<Smem<T, CONV>*>(smem_raw);
   constexpr bool kGate = HAS_Z && MODE == kFull;
 
   const int tid = threadIdx.x;
@@ -323,6 +334,33 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
     for (int n = 0; n < N; ++n) pamax = fmaxf(pamax, fabsf(p.A[dp * N + n] * kLog2e));
   }
   const float pclamp = kMaxDecayArg / fmaxf(pamax, 1e-30f);
+  // Convolution taps of channel pc, and (threads starting at step 0) the
+  // inputs just before this segment: from x itself past the first segment,
+  // else from conv_prev, else zero.  hist[i] is the input at step l0 - 3 + i.
+  const int K = CONV ? p.conv_width : 1;
+  float cw[kMaxConv] = {0.f, 0.f, 0.f, 0.f};  // cw[i] multiplies the input at t - 3 + i
+  float cbias = 0.f, hist[kMaxConv - 1] = {0.f, 0.f, 0.f};
+  if (CONV && d0 + pc < p.dim) {
+    const int64_t dp = d0 + pc;
+#pragma unroll
+    for (int i = 0; i < kMaxConv; ++i) {  // tap k = i - (kMaxConv - K) of the channel
+      const int k = i - (kMaxConv - K);
+      cw[i] = k >= 0 ? p.conv_w[dp * K + k] : 0.f;
+    }
+    cbias = p.conv_b ? p.conv_b[dp] : 0.f;
+    if (pt0 == 0) {
+      const T* xrow = static_cast<const T*>(p.u) + b * p.u_sb + dp * p.u_sd;
+#pragma unroll
+      for (int i = 0; i < kMaxConv - 1; ++i) {
+        const int64_t tt = l0 - (kMaxConv - 1) + i;  // step of hist[i]
+        if (tt >= 0 && tt < p.seqlen) {
+          hist[i] = to_f32<T>(xrow[tt]);
+        } else if (tt < 0 && p.conv_prev != nullptr && tt >= -(K - 1)) {
+          hist[i] = p.conv_prev[((b * p.dim + dp) * (K - 1)) + (K - 1) + tt];
+        }
+      }
+    }
+  }
 
   // ---- tile loads ----------------------------------------------------------------
   const int nch = static_cast<int>(imin64(kCH, p.dim - d0));  // valid channels
@@ -393,12 +431,44 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
       }
     }
     {  // dt' and dt' u of channel pc, steps [pt0, pt0 + 16)
+      // the convolution's window: three inputs before pt0 (the previous
+      // tile's last steps when pt0 = 0; that buffer is rewritten only after
+      // this prep)
+      float win[kMaxConv - 1];
+      if (CONV) {
+#pragma unroll
+        for (int i = 0; i < kMaxConv - 1; ++i) {
+          if (pt0 > 0) {
+            win[i] = to_f32<T>(sm.raw_u[ubuf][pc][pt0 - (kMaxConv - 1) + i]);
+          } else {
+            win[i] = k > 0 ? to_f32<T>(sm.raw_u[ubuf ^ 1][pc][kTL - (kMaxConv - 1) + i]) : hist[i];
+          }
+        }
+      }
 #pragma unroll
       for (int jj = 0; jj < kTL / kNG; jj += 8) {
         const int t = pt0 + jj;
         float dl[8], uv[8], vdt[8], vdu[8];
         load8<T>(&sm.raw_dl[pc][t], dl);
         load8<T>(&sm.raw_u[ubuf][pc][t], uv);
+        if (CONV) {  // uv <- silu(bias + sum_i cw[i] x[t - 3 + i])
+          float xs[kMaxConv - 1 + 8];
+#pragma unroll
+          for (int i = 0; i < kMaxConv - 1; ++i) xs[i] = win[i];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) xs[kMaxConv - 1 + i] = uv[i];
+#pragma unroll
+          for (int i = 0; i < kMaxConv - 1; ++i) win[i] = uv[8 - (kMaxConv - 1) + i];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float a = cbias;
+#pragma unroll
+            for (int tap = 0; tap < kMaxConv; ++tap) a = fmaf(cw[tap], xs[i + tap], a);
+            uv[i] = t + i < len ? gate_silu<T>(a) : 0.f;
+          }
+          *reinterpret_cast<float4*>(&sm.uc[pc][t]) = make_float4(uv[0], uv[1], uv[2], uv[3]);
+          *reinterpret_cast<float4*>(&sm.uc[pc][t + 4]) = make_float4(uv[4], uv[5], uv[6], uv[7]);
+        }
 #pragma unroll
         for (int q2 = 0; q2 < 8; q2 += 2) {
           float2 s = __fadd2_rn(make_float2(dl[q2], dl[q2 + 1]), make_float2(pbias, pbias));
@@ -493,7 +563,8 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
           acc.y = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);
         }
         if (yrow != nullptr && te < len) {
-          const float2 uv = load_pair<T>(&sm.raw_u[ubuf][cl][te]);
+          const float2 uv = CONV ? *reinterpret_cast<const float2*>(&sm.uc[cl][te])
+                                 : load_pair<T>(&sm.raw_u[ubuf][cl][te]);
           float y0 = fmaf(Dd, uv.x, acc.x);
           float y1 = fmaf(Dd, uv.y, acc.y);
           if (kGate) {

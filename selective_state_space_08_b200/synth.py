@@ -170,6 +170,19 @@ def make_scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str 
     return out
 
 
+def make_conv_params(dim: int, width: int = 4, seed: int = 9, batch: int | None = None,
+                     prev: bool = False) -> dict:
+    """Parameters of the convolution stage in front of the scan (float32):
+    weight (dim, width) ~ N(0, 1/width), bias (dim) ~ N(0, 0.1^2) and, with
+    ``prev``, a preceding window x_prev (batch, dim, width - 1) ~ N(0, 1)."""
+    rng = np.random.default_rng([seed, 7, width])
+    out = {"weight": (rng.standard_normal((dim, width)) / np.sqrt(width)).astype(np.float32),
+           "bias": (0.1 * rng.standard_normal(dim)).astype(np.float32), "x_prev": None}
+    if prev:
+        out["x_prev"] = rng.standard_normal((batch, dim, width - 1)).astype(np.float32)
+    return out
+
+
 def make_ssd_inputs(batch: int, seqlen: int, nheads: int, headdim: int, dstate: int,
                     dtype: str = "bf16", gate: bool = False, seed: int = 4,
                     s_range=(1e-3, 1e-1), h0: bool = False) -> dict:

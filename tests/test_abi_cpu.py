@@ -111,6 +111,22 @@ def test_host_scan_staging_and_host_side_errors(lib):
     assert lib.ssm_scan_fwd_host(ctypes.byref(_args(batch=0)), 1, None, 0, None) == 0
 
 
+def test_conv_scan_rejects_bad_stage_arguments(lib):
+    a = _args()
+    c = _abi.ConvArgs()
+    c.width, c.weight = 4, 0x10000
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(a), None, None, 0, None) == 1
+    for width in (0, 5):
+        c.width = width
+        assert lib.ssm_scan_fwd_conv(ctypes.byref(a), ctypes.byref(c), None, 0, None) == 2
+    c.width, c.weight = 4, None
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(a), ctypes.byref(c), None, 0, None) == 1
+    c.weight, c.bias = 0x10000, 0x10002
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(a), ctypes.byref(c), None, 0, None) == 3
+    c.bias = None
+    assert lib.ssm_scan_fwd_conv(ctypes.byref(_args(dim=0)), ctypes.byref(c), None, 0, None) == 0
+
+
 def _ssd_args(**kw):
     a = _abi.SsdArgs()
     a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.chunk = 2, 1000, 8, 64, 128, 256
