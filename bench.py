@@ -501,6 +501,24 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
                           "us_per_call": round(sec * 1e6, 3),
                           "GB_per_s": round(sbytes / sec / 1e9, 1),
                           "hbm_frac": round(sbytes / sec / 1e9 / hbm_peak, 4)}
+    # the same step, 64 steps per CUDA-graph replay (no per-call launch latency)
+    T = 64
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(T):
+            step()
+    total, per, _ = time_steps(graph.replay, max(3, steps // 8), warmup, flush, 1, None)
+    sec = total / max(3, steps // 8) / T
+    out["decode_step_graph"] = {"config": f"{out['decode_step']['config']}, {T} steps per graph replay",
+                                "us_per_call": round(sec * 1e6, 3),
+                                "GB_per_s": round(sbytes / sec / 1e9, 1),
+                                "hbm_frac": round(sbytes / sec / 1e9 / hbm_peak, 4)}
+    del graph
     return out
 
 
