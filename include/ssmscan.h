@@ -106,6 +106,14 @@ typedef struct {
   float* h_last;
   int64_t u_stride[2], delta_stride[2], z_stride[2], y_stride[2];
   int64_t B_stride[2], C_stride[2];
+  /* Grouped B and C: with ngroups > 1, B and C are (batch, ngroups, dstate,
+   * seqlen) and channel d reads group d / (dim / ngroups); dim / ngroups must
+   * be a multiple of 32 (SSM_ERR_UNSUPPORTED otherwise).  *_group_stride is
+   * the element stride between groups (0: the default dstate*seqlen); the
+   * default batch stride becomes ngroups*dstate*seqlen.  0 or 1: one group
+   * (the layout above).  Negative: SSM_ERR_INVALID_ARG. */
+  int64_t ngroups;
+  int64_t B_group_stride, C_group_stride;
 } ssm_scan_args_t;
 
 /* Bytes of scratch ssm_scan_fwd needs for these arguments (0 when the whole

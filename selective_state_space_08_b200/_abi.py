@@ -30,7 +30,8 @@ class ScanArgs(ctypes.Structure):
                 ("z", _vp), ("delta_bias", _fp), ("delta_softplus", ctypes.c_int),
                 ("h0", _fp), ("y", _vp), ("h_last", _fp),
                 ("u_stride", _i64 * 2), ("delta_stride", _i64 * 2), ("z_stride", _i64 * 2),
-                ("y_stride", _i64 * 2), ("B_stride", _i64 * 2), ("C_stride", _i64 * 2)]
+                ("y_stride", _i64 * 2), ("B_stride", _i64 * 2), ("C_stride", _i64 * 2),
+                ("ngroups", _i64), ("B_group_stride", _i64), ("C_group_stride", _i64)]
 
 
 class ConvArgs(ctypes.Structure):

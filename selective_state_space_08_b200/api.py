@@ -68,9 +68,12 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_las
     for name, t in (("delta", delta), ("z", z), ("y", y)):
         if t is not None and (t.dtype != dt or tuple(t.shape) != (batch, dim, L)):
             raise ValueError(f"{name} must be {dt} of shape {(batch, dim, L)}")
+    # B and C: (batch, N, L), or grouped (batch, groups, N, L)
+    G = B.shape[1] if B.dim() == 4 else 0
+    bc_shape = (batch, G, N, L) if G else (batch, N, L)
     for name, t in (("B", B), ("C", C)):
-        if t.dtype != dt or tuple(t.shape) != (batch, N, L):
-            raise ValueError(f"{name} must be {dt} of shape {(batch, N, L)}")
+        if t.dtype != dt or tuple(t.shape) != bc_shape:
+            raise ValueError(f"{name} must be {dt} of shape {bc_shape}")
     for name, t, shape in (("A", A, (dim, N)), ("D", D, (dim,)), ("delta_bias", delta_bias, (dim,)),
                            ("h0", h0, (batch, dim, N)), ("h_last", h_last, (batch, dim, N))):
         if t is not None:
@@ -87,9 +90,17 @@ def _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_las
     for field, name, t in (("u_stride", "u", u), ("delta_stride", "delta", delta), ("z_stride", "z", z),
                            ("y_stride", "y", y), ("B_stride", "B", B), ("C_stride", "C", C)):
         if t is not None and not host:
-            sb, sr = _seq_strides(name, t)
-            getattr(a, field)[0] = sb
-            getattr(a, field)[1] = sr
+            if t.dim() == 4:  # grouped: (batch, groups, N, L)
+                if t.shape[-1] > 1 and t.stride(-1) != 1:
+                    raise ValueError(f"{name} must be contiguous along the sequence")
+                getattr(a, field)[0] = t.stride(0)
+                getattr(a, field)[1] = t.stride(2)
+                setattr(a, f"{name}_group_stride", t.stride(1))
+            else:
+                sb, sr = _seq_strides(name, t)
+                getattr(a, field)[0] = sb
+                getattr(a, field)[1] = sr
+    a.ngroups = G
     return a
 
 

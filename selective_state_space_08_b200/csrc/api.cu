@@ -112,7 +112,13 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* out, bool check_ptrs 
   p.B = a->B;
   p.C = a->C;
   auto pick = [](int64_t s, int64_t def) { return s == 0 ? def : s; };
-  const int64_t xb = a->dim * L, xd = L, bcb = a->dstate * L, bcn = L;
+  if (a->ngroups < 0) return SSM_ERR_INVALID_ARG;
+  const int64_t G = a->ngroups > 1 ? a->ngroups : 1;
+  if (G > 1 && (a->dim % G != 0 || (a->dim / G) % fwd::kCH != 0)) return SSM_ERR_UNSUPPORTED;
+  p.group_ch = G > 1 ? a->dim / G : (a->dim > 0 ? a->dim : 1);
+  const int64_t xb = a->dim * L, xd = L, bcb = G * a->dstate * L, bcn = L;
+  p.B_sg = G > 1 ? pick(a->B_group_stride, a->dstate * L) : 0;
+  p.C_sg = G > 1 ? pick(a->C_group_stride, a->dstate * L) : 0;
   p.u_sb = pick(a->u_stride[0], xb);
   p.u_sd = pick(a->u_stride[1], xd);
   p.dl_sb = pick(a->delta_stride[0], xb);
@@ -125,8 +131,8 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* out, bool check_ptrs 
   p.B_sn = pick(a->B_stride[1], bcn);
   p.C_sb = pick(a->C_stride[0], bcb);
   p.C_sn = pick(a->C_stride[1], bcn);
-  const int64_t strides[] = {p.u_sb, p.u_sd, p.dl_sb, p.dl_sd, p.z_sb, p.z_sd,
-                             p.y_sb, p.y_sd, p.B_sb, p.B_sn, p.C_sb, p.C_sn};
+  const int64_t strides[] = {p.u_sb, p.u_sd, p.dl_sb, p.dl_sd, p.z_sb, p.z_sd, p.y_sb,
+                             p.y_sd, p.B_sb, p.B_sn, p.C_sb, p.C_sn, p.B_sg, p.C_sg};
   for (int64_t s : strides)
     if (s < 0) return SSM_ERR_INVALID_ARG;
   p.A = a->A;
@@ -438,6 +444,7 @@ ssm_status_t plan_host(const ssm_scan_args_t* a, int64_t sb, HostPlan* hp) {
                               a->y_stride, a->B_stride, a->C_stride};
   for (const int64_t* st : strides)
     if (st[0] != 0 || st[1] != 0) return SSM_ERR_UNSUPPORTED;
+  if (a->B_group_stride != 0 || a->C_group_stride != 0) return SSM_ERR_UNSUPPORTED;
   ScanPlan whole;
   ssm_status_t st = plan_scan(a, &whole);  // sizes, flags and the host pointers
   if (st != SSM_OK) return st;
@@ -456,10 +463,11 @@ ssm_status_t plan_host(const ssm_scan_args_t* a, int64_t sb, HostPlan* hp) {
   }
   const size_t es = elem_size(a->dtype);
   const size_t D = static_cast<size_t>(a->dim), N = static_cast<size_t>(a->dstate);
+  const size_t NB = N * static_cast<size_t>(a->ngroups > 1 ? a->ngroups : 1);  // B/C rows per batch
   const size_t L = static_cast<size_t>(a->seqlen), S = static_cast<size_t>(hp->sb);
   hp->es = es;
   hp->x_bytes = S * D * L * es;
-  hp->bc_bytes = S * N * L * es;
+  hp->bc_bytes = S * NB * L * es;
   hp->h_bytes = S * D * N * sizeof(float);
   size_t o = 0;
   hp->off_A = o;    o += round256(D * N * sizeof(float));
@@ -530,6 +538,7 @@ ssm_status_t run_host(const ssm_scan_args_t* a, const HostPlan& hp, unsigned cha
                          "scan_fwd_host: copy to host");
   };
   const size_t D = static_cast<size_t>(a->dim), N = static_cast<size_t>(a->dstate);
+  const size_t NB = N * static_cast<size_t>(a->ngroups > 1 ? a->ngroups : 1);  // B/C rows per batch
   const size_t L = static_cast<size_t>(a->seqlen), es = hp.es;
   if (st == SSM_OK && chk(cudaEventRecord(ev_start, stream), "scan_fwd_host: record") &&
       chk(cudaStreamWaitEvent(sin, ev_start, 0), "scan_fwd_host: wait") &&
@@ -543,7 +552,7 @@ ssm_status_t run_host(const ssm_scan_args_t* a, const HostPlan& hp, unsigned cha
       const int64_t b0 = s * hp.sb;
       const int64_t nb = a->batch - b0 < hp.sb ? a->batch - b0 : hp.sb;
       const size_t xo = static_cast<size_t>(b0) * D * L * es, xn = static_cast<size_t>(nb) * D * L * es;
-      const size_t bo = static_cast<size_t>(b0) * N * L * es, bn = static_cast<size_t>(nb) * N * L * es;
+      const size_t bo = static_cast<size_t>(b0) * NB * L * es, bn = static_cast<size_t>(nb) * NB * L * es;
       const size_t ho = static_cast<size_t>(b0) * D * N * sizeof(float);
       const size_t hn = static_cast<size_t>(nb) * D * N * sizeof(float);
       auto in = [](const void* base, size_t off) {

@@ -55,6 +55,8 @@ struct ScanParams {
   const void* B;
   const void* C;
   int64_t u_sb, u_sd, dl_sb, dl_sd, z_sb, z_sd, y_sb, y_sd, B_sb, B_sn, C_sb, C_sn;
+  int64_t B_sg, C_sg;  // stride between groups of B / C
+  int64_t group_ch;    // channels per group (dim when B and C are not grouped)
   const float* A;
   const float* D;
   const float* bias;
@@ -366,8 +368,9 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
   const int nch = static_cast<int>(imin64(kCH, p.dim - d0));  // valid channels
   const T* tu = gu + b * p.u_sb + d0 * p.u_sd;
   const T* tdl = gdl + b * p.dl_sb + d0 * p.dl_sd;
-  const T* tB = gB + b * p.B_sb;
-  const T* tC = gC + b * p.C_sb;
+  const int64_t grp = d0 / p.group_ch;  // a block's channels share one group
+  const T* tB = gB + b * p.B_sb + grp * p.B_sg;
+  const T* tC = gC + b * p.C_sb + grp * p.C_sg;
   auto issue_load = [&](int ubuf, int64_t t0) {
     const int len = static_cast<int>(imin64(kTL, l1 - t0));
     if (VEC) {

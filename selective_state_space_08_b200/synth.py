@@ -170,6 +170,16 @@ def make_scan_inputs(batch: int, dim: int, dstate: int, seqlen: int, dtype: str 
     return out
 
 
+def make_grouped_bc(batch: int, ngroups: int, dstate: int, seqlen: int, dtype: str = "bf16",
+                    seed: int = 5) -> dict:
+    """Grouped B and C, (batch, ngroups, dstate, seqlen) ~ N(0, 1), rounded to
+    ``dtype`` (float32 arrays)."""
+    rng = np.random.default_rng([seed, 11, ngroups])
+    shape = (batch, ngroups, dstate, seqlen)
+    return {"B": round_to(rng.standard_normal(shape).astype(np.float32), dtype),
+            "C": round_to(rng.standard_normal(shape).astype(np.float32), dtype)}
+
+
 def make_conv_params(dim: int, width: int = 4, seed: int = 9, batch: int | None = None,
                      prev: bool = False) -> dict:
     """Parameters of the convolution stage in front of the scan (float32):

@@ -111,6 +111,15 @@ def test_host_scan_staging_and_host_side_errors(lib):
     assert lib.ssm_scan_fwd_host(ctypes.byref(_args(batch=0)), 1, None, 0, None) == 0
 
 
+def test_grouped_bc_arguments(lib):
+    """Groups must hold whole 32-channel blocks; a negative count is invalid."""
+    ok = _args(dim=64, ngroups=2)
+    assert lib.ssm_scan_fwd_workspace_size(ctypes.byref(ok)) != ctypes.c_size_t(-1).value
+    assert lib.ssm_scan_fwd(ctypes.byref(_args(dim=40, ngroups=2)), None, 0, None) == 2
+    assert lib.ssm_scan_fwd(ctypes.byref(_args(dim=96, ngroups=2)), None, 0, None) == 2
+    assert lib.ssm_scan_fwd(ctypes.byref(_args(ngroups=-1)), None, 0, None) == 1
+
+
 def test_conv_scan_rejects_bad_stage_arguments(lib):
     a = _args()
     c = _abi.ConvArgs()
