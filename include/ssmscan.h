@@ -155,6 +155,24 @@ typedef struct {
 ssm_status_t ssm_scan_fwd_conv(const ssm_scan_args_t* args, const ssm_conv_args_t* conv,
                                void* workspace, size_t workspace_bytes, ssm_stream_t stream);
 
+/* The selective scan over a packed variable-length batch: nseq sequences
+ * laid end to end along seqlen in one batch row (args->batch must be 1),
+ * sequence i covering steps [cu_seqlens[i], cu_seqlens[i+1]).  The state
+ * restarts from zero at every sequence start, and h_last (if not NULL) is
+ * (nseq, dim, dstate) fp32: the state after each sequence's last step.
+ *   cu_seqlens : device int32 (nseq + 1), cu_seqlens[0] = 0, strictly
+ *                increasing (every sequence non-empty), cu_seqlens[nseq] =
+ *                seqlen; other contents give undefined results (no
+ *                out-of-bounds access).
+ * args->h0 must be NULL (SSM_ERR_UNSUPPORTED otherwise); the rest of `args`
+ * as for ssm_scan_fwd.  Workspace: ssm_scan_fwd_workspace_size(args).
+ * Page "Mamba状态空间模型的硬件感知推理优化" section 1 and page
+ * "从硬件感知到算法革命" (dynamic batching): each sequence is an independent
+ * recurrence; packing only shares the launch. */
+ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_args_t* args, const int32_t* cu_seqlens,
+                                 int64_t nseq, void* workspace, size_t workspace_bytes,
+                                 ssm_stream_t stream);
+
 /* Bytes of the library's static device scratch used by ssm_scan_fwd_noalloc. */
 #define SSM_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 

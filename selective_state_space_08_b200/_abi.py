@@ -81,6 +81,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_scan_fwd_conv.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ConvArgs), _vp,
                                       ctypes.c_size_t, _vp]
     lib.ssm_scan_fwd_conv.restype = ctypes.c_int
+    lib.ssm_scan_fwd_varlen.argtypes = [ctypes.POINTER(ScanArgs), _vp, _i64, _vp, ctypes.c_size_t,
+                                        _vp]
+    lib.ssm_scan_fwd_varlen.restype = ctypes.c_int
     lib.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _vp]
     lib.ssm_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_scan_fwd_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), _i64]

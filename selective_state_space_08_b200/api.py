@@ -188,6 +188,44 @@ def scan_fwd_conv(x, conv_weight, conv_bias, x_prev, delta, A, B, C, D=None, z=N
     return y, h_last
 
 
+def scan_fwd_varlen(u, delta, A, B, C, cu_seqlens, D=None, z=None, delta_bias=None,
+                    delta_softplus=True, *, y=None, h_last=None, return_last_state=True,
+                    workspace=None, stream=None):
+    """Selective scan over a packed variable-length batch: u, delta, z are
+    (1, dim, L) and B, C (1, N, L) (or grouped), holding the sequences end to
+    end; cu_seqlens: int32 CUDA tensor (nseq + 1) of sequence offsets.  Each
+    sequence starts from a zero state.  Returns (y, h_last (nseq, dim, N))."""
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+                    ("delta_bias", delta_bias), ("y", y), ("h_last", h_last)):
+        _cuda(name, t)
+    _cuda("cu_seqlens", cu_seqlens, torch.int32, 1)
+    if not cu_seqlens.is_contiguous() or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be a contiguous int32 vector of nseq + 1 offsets")
+    if u.dim() != 3 or u.shape[0] != 1:
+        raise ValueError("u must be (1, dim, L)")
+    nseq = cu_seqlens.numel() - 1
+    dim, N = u.shape[1], A.shape[1]
+    if y is None:
+        y = torch.empty(u.shape, dtype=u.dtype, device=u.device)
+    if h_last is None and return_last_state:
+        h_last = torch.empty((nseq, dim, N), dtype=torch.float32, device=u.device)
+    if h_last is not None and (h_last.dtype != torch.float32 or tuple(h_last.shape) != (nseq, dim, N)
+                               or not h_last.is_contiguous()):
+        raise ValueError(f"h_last must be contiguous float32 of shape {(nseq, dim, N)}")
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, None, y, None)
+    a.h_last = _ptr(h_last)
+    lib = _abi.load()
+    need = lib.ssm_scan_fwd_workspace_size(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(int(need), dtype=torch.uint8, device=u.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _abi.check(lib.ssm_scan_fwd_varlen(ctypes.byref(a), _ptr(cu_seqlens), nseq, _ptr(workspace),
+                                       ws_bytes, _stream(stream)), "ssm_scan_fwd_varlen")
+    return y, h_last
+
+
 def scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                      h0=None, *, y, h_last=None, stream=None):
     """``scan_fwd`` for callers that cannot allocate device memory: ``y`` (and

@@ -177,9 +177,9 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* out, bool check_ptrs 
   return SSM_OK;
 }
 
-template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV>
+template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV, bool VARLEN>
 ssm_status_t launch_fwd(const ScanParams& p, cudaStream_t stream) {
-  auto kernel = fwd::scan_fwd_kernel<T, MODE, HAS_Z, VEC, CONV>;
+  auto kernel = fwd::scan_fwd_kernel<T, MODE, HAS_Z, VEC, CONV, VARLEN>;
   const size_t smem = sizeof(fwd::Smem<T, CONV>);
   ssm_status_t st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem),
                                 "scan_fwd: shared-memory opt-in");
@@ -192,11 +192,11 @@ ssm_status_t launch_fwd(const ScanParams& p, cudaStream_t stream) {
                                                            : "scan_fwd: scan pass launch");
 }
 
-template <typename T, bool VEC, bool CONV>
+template <typename T, bool VEC, bool CONV, bool VARLEN = false>
 ssm_status_t run_fwd(const ScanParams& p, cudaStream_t stream) {
   ssm_status_t st = SSM_OK;
   if (p.nseg > 1) {
-    st = launch_fwd<T, fwd::kAgg, false, VEC, CONV>(p, stream);
+    st = launch_fwd<T, fwd::kAgg, false, VEC, CONV, VARLEN>(p, stream);
     if (st != SSM_OK) return st;
     const int64_t total = p.batch * p.dim * fwd::kMaxN;
     const int threads = 256;
@@ -205,8 +205,8 @@ ssm_status_t run_fwd(const ScanParams& p, cudaStream_t stream) {
     st = cuda_status(cudaGetLastError(), "scan_fwd: carry launch");
     if (st != SSM_OK) return st;
   }
-  return p.z != nullptr ? launch_fwd<T, fwd::kFull, true, VEC, CONV>(p, stream)
-                        : launch_fwd<T, fwd::kFull, false, VEC, CONV>(p, stream);
+  return p.z != nullptr ? launch_fwd<T, fwd::kFull, true, VEC, CONV, VARLEN>(p, stream)
+                        : launch_fwd<T, fwd::kFull, false, VEC, CONV, VARLEN>(p, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -602,15 +602,19 @@ ssm_status_t run_host(const ssm_scan_args_t* a, const HostPlan& hp, unsigned cha
   return st;
 }
 
-// ssm_scan_fwd, with the convolution stage in front when `conv` is given.
+// ssm_scan_fwd, with the convolution stage in front when `conv` is given,
+// or over a packed variable-length batch when `cu_seqlens` is.
 ssm_status_t scan_fwd_impl(const ssm_scan_args_t* args, const ssm_conv_args_t* conv,
-                           void* workspace, size_t workspace_bytes, ssm_stream_t stream_) {
+                           void* workspace, size_t workspace_bytes, ssm_stream_t stream_,
+                           const int32_t* cu_seqlens = nullptr, int64_t nseq = 0) {
   ScanPlan plan;
   ssm_status_t st = plan_scan(args, &plan);
   if (st != SSM_OK) return st;
   ScanParams& p = plan.p;
   p.conv_width = 0;
   p.conv_w = p.conv_b = p.conv_prev = nullptr;
+  p.cu_seqlens = cu_seqlens;
+  p.nseq = nseq;
   if (conv != nullptr) {
     if (conv->width < 1 || conv->width > fwd::kMaxConv) return SSM_ERR_UNSUPPORTED;
     if (p.batch > 0 && p.dim > 0 && conv->weight == nullptr) return SSM_ERR_INVALID_ARG;
@@ -636,6 +640,13 @@ ssm_status_t scan_fwd_impl(const ssm_scan_args_t* args, const ssm_conv_args_t* c
   }
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   const bool bf16 = args->dtype == SSM_BF16;
+  if (cu_seqlens != nullptr) {
+    if (bf16)
+      return plan.vec ? run_fwd<__nv_bfloat16, true, false, true>(p, stream)
+                      : run_fwd<__nv_bfloat16, false, false, true>(p, stream);
+    return plan.vec ? run_fwd<float, true, false, true>(p, stream)
+                    : run_fwd<float, false, false, true>(p, stream);
+  }
   if (conv != nullptr) {
     if (bf16)
       return plan.vec ? run_fwd<__nv_bfloat16, true, true>(p, stream)
@@ -667,6 +678,16 @@ ssm_status_t ssm_scan_fwd_conv(const ssm_scan_args_t* args, const ssm_conv_args_
                                void* workspace, size_t workspace_bytes, ssm_stream_t stream) {
   if (conv == nullptr) return SSM_ERR_INVALID_ARG;
   return scan_fwd_impl(args, conv, workspace, workspace_bytes, stream);
+}
+
+ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_args_t* args, const int32_t* cu_seqlens,
+                                 int64_t nseq, void* workspace, size_t workspace_bytes,
+                                 ssm_stream_t stream) {
+  if (args == nullptr || cu_seqlens == nullptr || nseq < 1) return SSM_ERR_INVALID_ARG;
+  if (args->batch != 1 || args->h0 != nullptr || args->seqlen > INT32_MAX)
+    return SSM_ERR_UNSUPPORTED;
+  if (!aligned(cu_seqlens, 4)) return SSM_ERR_ALIGNMENT;
+  return scan_fwd_impl(args, nullptr, workspace, workspace_bytes, stream, cu_seqlens, nseq);
 }
 
 size_t ssm_scan_fwd_host_staging_size(const ssm_scan_args_t* args, int64_t slice_batch) {

@@ -72,6 +72,11 @@ struct ScanParams {
   const float* conv_w;      // (dim, conv_width)
   const float* conv_b;      // (dim) or null
   const float* conv_prev;   // (batch, dim, conv_width - 1) inputs before step 0, or null
+  // Packed variable-length batch (batch 1): sequence i covers steps
+  // [cu_seqlens[i], cu_seqlens[i + 1]); the state restarts from zero at each
+  // start, and h_last is (nseq, dim, dstate), one state per sequence.
+  const int32_t* cu_seqlens;
+  int64_t nseq;
 };
 
 namespace fwd {
@@ -110,6 +115,10 @@ struct Smem {
   // convolution output u (fp32) for the epilogue's skip term; rows of 72
   // floats put the epilogue's 8-byte reads on distinct banks
   float uc[CONV ? kCH : 1][kTL + 8];
+  // packed batches: the tile's sequence starts and last steps (bit t = step
+  // t0 + t) and the sequence that contains step t0
+  unsigned long long vl_start, vl_end;
+  long long vl_seq;
 };
 
 constexpr int kMaxConv = 4;  // taps of the convolution stage
@@ -279,7 +288,7 @@ __device__ __forceinline__ void sub_decays(const float* dtp_row, float2 A01, flo
   }
 }
 
-template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV = false>
+template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV = false, bool VARLEN = false>
 __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem<T, CONV>& sm = *reinterpret_cast<Smem<T, CONV>*>(smem_raw);
@@ -323,6 +332,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
   float2 h23 = make_float2(hin[2], hin[3]);
   const float Dd = (ch_ok && p.D) ? p.D[d] : 0.f;
   float dtsum = 0.f;
+  bool restarted = false;  // packed batches: a sequence starts inside this segment
   const T* zrow = kGate && ch_ok ? static_cast<const T*>(p.z) + b * p.z_sb + d * p.z_sd : nullptr;
   T* yrow = MODE == kFull && ch_ok ? static_cast<T*>(p.y) + b * p.y_sb + d * p.y_sd : nullptr;
 
@@ -417,6 +427,23 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
     __syncthreads();  // tile k visible; every thread is done with tile k - 1
 
     // ---- per-tile preparation ------------------------------------------------------
+    if (VARLEN && tid == 0) {  // sequence starts / last steps inside [t0, t0 + len)
+      const int32_t* cu = p.cu_seqlens;
+      int64_t lo = 0, hi = p.nseq - 1;  // the last sequence starting at or before t0
+      while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) / 2;
+        if (cu[mid] <= t0) lo = mid; else hi = mid - 1;
+      }
+      unsigned long long st = 0ull, en = 0ull;
+      for (int64_t i = lo; i < p.nseq && cu[i] < t0 + len; ++i) {
+        const int64_t s0 = cu[i], e0 = static_cast<int64_t>(cu[i + 1]) - 1;
+        if (s0 >= t0) st |= 1ull << (s0 - t0);
+        if (e0 >= t0 && e0 < t0 + len) en |= 1ull << (e0 - t0);
+      }
+      sm.vl_start = st;
+      sm.vl_end = en;
+      sm.vl_seq = lo;
+    }
     {  // B and C to fp32, [step][state]: thread -> states 4q .. 4q+3, steps r and r + 32
       static_assert(kThreads == 128 && kTL == 64 && kMaxN == 16, "prep mapping");
       const int r = tid % 32;
@@ -504,6 +531,9 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
     }
     const float* bf = &sm.Bf[0][kNPT * g];
     const float* cf = &sm.Cf[0][kNPT * g];
+    const unsigned long long vstart = VARLEN ? sm.vl_start : 0ull;
+    const unsigned long long vend = VARLEN ? sm.vl_end : 0ull;
+    if (VARLEN && vstart != 0ull) restarted = true;
     // Every sub-tile of the tile is processed (steps past `len` carry dt' = 0 and
     // dt' u = 0, which leave the state unchanged), so the loop unrolls fully.
     // The decays of sub-tile s + 1 are computed while sub-tile s runs its
@@ -526,8 +556,22 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
         const int t = tb + tt;
         const float4 bq = *reinterpret_cast<const float4*>(bf + t * kBCRow);
         const float2 du2 = make_float2(dus[tt], dus[tt]);
-        h01 = __ffma2_rn(dcur.a01[tt], h01, __fmul2_rn(du2, make_float2(bq.x, bq.y)));
-        h23 = __ffma2_rn(dcur.a23[tt], h23, __fmul2_rn(du2, make_float2(bq.z, bq.w)));
+        float2 a01 = dcur.a01[tt], a23 = dcur.a23[tt];
+        if (VARLEN && ((vstart >> t) & 1ull)) a01 = a23 = make_float2(0.f, 0.f);  // restart
+        h01 = __ffma2_rn(a01, h01, __fmul2_rn(du2, make_float2(bq.x, bq.y)));
+        h23 = __ffma2_rn(a23, h23, __fmul2_rn(du2, make_float2(bq.z, bq.w)));
+        if (VARLEN && MODE == kFull && ((vend >> t) & 1ull) && ch_ok && p.h_last != nullptr) {
+          // the last step of a sequence: its state goes to h_last[sequence]
+          const unsigned long long upto = t == 63 ? ~0ull : ((2ull << t) - 1ull);
+          int64_t sq = sm.vl_seq + __popcll(vstart & upto & ~1ull);
+          sq = sq < 0 ? 0 : (sq >= p.nseq ? p.nseq - 1 : sq);
+          const float hv[kNPT] = {h01.x, h01.y, h23.x, h23.y};
+#pragma unroll
+          for (int kk = 0; kk < kNPT; ++kk) {
+            const int n = g * kNPT + kk;
+            if (n < N) p.h_last[(sq * p.dim + d) * N + n] = hv[kk];
+          }
+        }
         if (MODE == kFull) {
           const float4 cq = *reinterpret_cast<const float4*>(cf + t * kBCRow);
           float2 yv = __fmul2_rn(make_float2(cq.x, cq.y), h01);
@@ -591,7 +635,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
   if (!ch_ok) return;
   const float hs[kNPT] = {h01.x, h01.y, h23.x, h23.y};
   if (MODE == kFull) {
-    if (p.h_last != nullptr && seg == p.nseg - 1) {
+    if (!VARLEN && p.h_last != nullptr && seg == p.nseg - 1) {
 #pragma unroll
       for (int kk = 0; kk < kNPT; ++kk) {
         const int n = g * kNPT + kk;
@@ -602,7 +646,8 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
     const int64_t slot = seg * p.batch * p.dim + bd;
 #pragma unroll
     for (int kk = 0; kk < kNPT; ++kk) p.carry_h[slot * kMaxN + g * kNPT + kk] = hs[kk];
-    if (g == 0) p.carry_dt[slot] = dtsum;
+    // a restart inside the segment cuts off the state entering it
+    if (g == 0) p.carry_dt[slot] = restarted ? __int_as_float(0x7f800000) : dtsum;
   }
 }
 
@@ -622,7 +667,8 @@ __global__ void scan_carry_kernel(const ScanParams p) {
   float hs = p.h0 ? p.h0[bd * N + n] : 0.f;
   for (int64_t s = 0; s + 1 < p.nseg; ++s) {
     const int64_t slot = s * p.batch * p.dim + bd;
-    hs = fmaf(expf(a * p.carry_dt[slot]), hs, p.carry_h[slot * kMaxN + n]);
+    const float dts = p.carry_dt[slot];  // +inf: a sequence restarted inside segment s
+    hs = fmaf(isinf(dts) ? 0.f : expf(a * dts), hs, p.carry_h[slot * kMaxN + n]);
     p.carry_h[slot * kMaxN + n] = hs;
   }
 }

@@ -120,6 +120,17 @@ def test_grouped_bc_arguments(lib):
     assert lib.ssm_scan_fwd(ctypes.byref(_args(ngroups=-1)), None, 0, None) == 1
 
 
+def test_varlen_scan_host_checks(lib):
+    cu = 0x10000  # never dereferenced: every case below fails on the host
+    a = _args(batch=1)
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(a), None, 2, None, 0, None) == 1
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(a), cu, 0, None, 0, None) == 1
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(_args(batch=2)), cu, 2, None, 0, None) == 2
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(_args(batch=1, h0=0x10000)), cu, 2, None, 0,
+                                   None) == 2
+    assert lib.ssm_scan_fwd_varlen(ctypes.byref(a), 0x10002, 2, None, 0, None) == 3
+
+
 def test_conv_scan_rejects_bad_stage_arguments(lib):
     a = _args()
     c = _abi.ConvArgs()
