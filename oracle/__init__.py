@@ -64,6 +64,9 @@ def _bind(lib):
     lib.oracle_ssd_fwd.argtypes = [_i64] * 5 + [_dp] * 8 + [ctypes.c_int, _dp, _dp, _dp,
                                                             ctypes.c_int]
     lib.oracle_ssd_fwd.restype = ctypes.c_int
+    lib.oracle_scan_bwd.argtypes = ([_i64] * 4 + [_dp] * 8 + [ctypes.c_int] + [_dp] * 2 +
+                                    [_dp] * 9)
+    lib.oracle_scan_bwd.restype = ctypes.c_int
     lib.oracle_conv_silu.argtypes = [_i64] * 4 + [_dp] * 5 + [ctypes.c_int]
     lib.oracle_conv_silu.restype = ctypes.c_int
     return lib
@@ -111,6 +114,45 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     if rc != 0:
         raise RuntimeError(f"oracle_scan_fwd failed ({rc})")
     return y, h_last
+
+
+def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=True,
+             h0=None, lib=None):
+    """Gradients of sum(y * dy) for the selective scan.  Shapes as in
+    ``scan_fwd``; dy like y.  Returns a dict of float64 arrays: du, ddelta,
+    dA, dB, dC, and (when the matching input is given) dD, dz, ddelta_bias,
+    dh0."""
+    u = _f64(u)
+    batch, dim, L = u.shape
+    N = np.asarray(A).shape[1]
+    delta = _f64(delta, u.shape)
+    A = _f64(A, (dim, N))
+    B = _f64(B, (batch, N, L))
+    C = _f64(C, (batch, N, L))
+    D = _f64(D, (dim,))
+    z = _f64(z, u.shape)
+    delta_bias = _f64(delta_bias, (dim,))
+    h0 = _f64(h0, (batch, dim, N))
+    dy = _f64(dy, u.shape)
+    out = {"du": np.zeros(u.shape), "ddelta": np.zeros(u.shape), "dA": np.zeros((dim, N)),
+           "dB": np.zeros((batch, N, L)), "dC": np.zeros((batch, N, L))}
+    if D is not None:
+        out["dD"] = np.zeros(dim)
+    if z is not None:
+        out["dz"] = np.zeros(u.shape)
+    if delta_bias is not None:
+        out["ddelta_bias"] = np.zeros(dim)
+    if h0 is not None:
+        out["dh0"] = np.zeros((batch, dim, N))
+    lib = lib or load()
+    g = lambda k: _p(out.get(k))
+    rc = lib.oracle_scan_bwd(batch, dim, N, L, _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(z),
+                             _p(delta_bias), int(bool(delta_softplus)), _p(h0), _p(dy), g("du"),
+                             g("ddelta"), g("dA"), g("dB"), g("dC"), g("dD"), g("dz"),
+                             g("ddelta_bias"), g("dh0"))
+    if rc != 0:
+        raise RuntimeError(f"oracle_scan_bwd failed ({rc})")
+    return out
 
 
 def conv_silu(x, w, bias=None, x_prev=None, nthreads=None, lib=None):

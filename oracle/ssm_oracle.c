@@ -294,4 +294,91 @@ int oracle_conv_silu(int64_t batch, int64_t dim, int64_t seqlen, int64_t width, 
   return 0;
 }
 
-int oracle_abi_version(void) { return 2; }
+/* ------------------------------------------------------------------ */
+/* Gradients of the selective scan (reverse mode), for a loss whose gradient
+ * with respect to y is dy.  [P2] section 1 ("recomputation": intermediate
+ * states are rebuilt in the backward pass instead of stored) -- here the
+ * states of one channel are simply recomputed in full, in order, before the
+ * reverse sweep.  With s_t = sum_n C[t,n] h[t,n] + D u_t and y_t = s_t g_t,
+ * g_t = silu(z_t) (1 without z), the adjoint of the recurrence is
+ *   lambda[t,n] = ds_t C[t,n] + dA[t+1,n] lambda[t+1,n],  ds_t = dy_t g_t,
+ * and every input receives the terms of the chain rule through dt'_t,
+ * dA[t,n] = exp(dt'_t A[n]) and dt'_t B[t,n] u_t.  Single-threaded (B and C
+ * gradients are sums over channels).  Outputs are overwritten; any of them
+ * may be NULL.  Shapes as in oracle_scan_fwd; dA (dim, dstate), dD, dbias
+ * (dim), dh0 (batch, dim, dstate). */
+static double softplus_grad(double s) { return s > 20.0 ? 1.0 : 1.0 / (1.0 + exp(-s)); }
+
+int oracle_scan_bwd(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen, const double* u,
+                    const double* delta, const double* A, const double* B, const double* C,
+                    const double* D, const double* z, const double* bias, int softplus,
+                    const double* h0, const double* dy, double* du, double* ddelta, double* dA,
+                    double* dB, double* dC, double* dD, double* dz, double* dbias, double* dh0) {
+  if (batch < 0 || dim < 0 || dstate < 0 || seqlen < 0) return -1;
+  const int64_t N = dstate, L = seqlen;
+  if (dA) for (int64_t i = 0; i < dim * N; ++i) dA[i] = 0.0;
+  if (dB) for (int64_t i = 0; i < batch * N * L; ++i) dB[i] = 0.0;
+  if (dC) for (int64_t i = 0; i < batch * N * L; ++i) dC[i] = 0.0;
+  if (dD) for (int64_t i = 0; i < dim; ++i) dD[i] = 0.0;
+  if (dbias) for (int64_t i = 0; i < dim; ++i) dbias[i] = 0.0;
+  double* hs = (double*)malloc(sizeof(double) * (size_t)((L + 1) * (N > 0 ? N : 1)));
+  double* dts = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+  double* lam = (double*)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+  for (int64_t row = 0; row < batch * dim; ++row) {
+    const int64_t b = row / dim, d = row % dim;
+    const double* ur = u + row * L;
+    const double* dl = delta + row * L;
+    const double* Bb = B + b * N * L;
+    const double* Cb = C + b * N * L;
+    const double* Ad = A + d * N;
+    /* forward: hs[(t + 1) N + n] = h[t, n], hs[n] = h0 */
+    for (int64_t n = 0; n < N; ++n) hs[n] = h0 ? h0[row * N + n] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+      const double dt = step_size(dl[t], bias, d, softplus);
+      dts[t] = dt;
+      for (int64_t n = 0; n < N; ++n)
+        hs[(t + 1) * N + n] = exp(dt * Ad[n]) * hs[t * N + n] + dt * Bb[n * L + t] * ur[t];
+    }
+    /* reverse sweep */
+    for (int64_t n = 0; n < N; ++n) lam[n] = 0.0;
+    double dDd = 0.0, dbd = 0.0;
+    for (int64_t t = L - 1; t >= 0; --t) {
+      const double dt = dts[t];
+      double sv = D ? D[d] * ur[t] : 0.0;
+      for (int64_t n = 0; n < N; ++n) sv += Cb[n * L + t] * hs[(t + 1) * N + n];
+      double gate = 1.0, ds = dy[row * L + t];
+      if (z) {
+        const double zv = z[row * L + t], sg = 1.0 / (1.0 + exp(-zv));
+        gate = zv * sg;
+        if (dz) dz[row * L + t] = dy[row * L + t] * sv * (sg * (1.0 + zv * (1.0 - sg)));
+      }
+      ds *= gate;
+      double du_t = D ? ds * D[d] : 0.0, ddt = 0.0;
+      dDd += ds * ur[t];
+      for (int64_t n = 0; n < N; ++n) {
+        lam[n] += ds * Cb[n * L + t];                     /* lambda_t = ds C_t + dA_{t+1} lambda_{t+1} */
+        const double a = exp(dt * Ad[n]), hp = hs[t * N + n];
+        if (dC) dC[b * N * L + n * L + t] += ds * hs[(t + 1) * N + n];
+        if (dB) dB[b * N * L + n * L + t] += lam[n] * dt * ur[t];
+        du_t += lam[n] * dt * Bb[n * L + t];
+        ddt += lam[n] * (Ad[n] * a * hp + Bb[n * L + t] * ur[t]);
+        if (dA) dA[d * N + n] += lam[n] * dt * a * hp;
+        lam[n] *= a;                                      /* carried to step t - 1 */
+      }
+      if (du) du[row * L + t] = du_t;
+      const double sarg = dl[t] + (bias ? bias[d] : 0.0);
+      const double dd = softplus ? ddt * softplus_grad(sarg) : ddt;
+      if (ddelta) ddelta[row * L + t] = dd;
+      dbd += dd;
+    }
+    if (dh0) for (int64_t n = 0; n < N; ++n) dh0[row * N + n] = lam[n];
+    if (dD) dD[d] += dDd;
+    if (dbias) dbias[d] += dbd;
+  }
+  free(hs);
+  free(dts);
+  free(lam);
+  return 0;
+}
+
+int oracle_abi_version(void) { return 3; }

@@ -483,9 +483,51 @@ def pin_conv_feeds_scan(lib):
     _close(h, hr, what="conv feeding the scan: h_L")
 
 
+# ---- gradients (reverse mode) -----------------------------------------------------
+
+
+def pin_backward_finite_differences(lib):
+    """G1: every gradient of the backward oracle equals the central finite
+    difference of sum(y * dy) computed with the (separately pinned) forward
+    oracle, on sampled entries of every input, with and without softplus."""
+    rng = np.random.default_rng(41)
+    for softplus in (True, False):
+        inp = _rand_scan(rng, batch=2, dim=3, N=4, L=9)
+        if not softplus:  # keep dt' = delta + bias positive and moderate
+            inp["delta"] = np.abs(inp["delta"]) * 0.3
+            inp["delta_bias"] = np.full(3, 0.05)
+        dy = rng.standard_normal(inp["u"].shape)
+        names = ["u", "delta", "A", "B", "C", "D", "z", "delta_bias", "h0"]
+
+        def loss(vals):
+            y, _ = oracle.scan_fwd(vals["u"], vals["delta"], vals["A"], vals["B"], vals["C"],
+                                   vals["D"], vals["z"], vals["delta_bias"], softplus, vals["h0"],
+                                   lib=lib)
+            return float(np.sum(y * dy))
+
+        g = oracle.scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, inp["D"],
+                            inp["z"], inp["delta_bias"], softplus, inp["h0"], lib=lib)
+        key = {"u": "du", "delta": "ddelta", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+               "z": "dz", "delta_bias": "ddelta_bias", "h0": "dh0"}
+        for name in names:
+            grad = g[key[name]]
+            flat = inp[name].reshape(-1)
+            for idx in rng.choice(flat.size, size=min(6, flat.size), replace=False):
+                eps = 1e-5 * max(1.0, abs(flat[idx]))
+                plus = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in inp.items()}
+                minus = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in inp.items()}
+                plus[name].reshape(-1)[idx] += eps
+                minus[name].reshape(-1)[idx] -= eps
+                fd = (loss(plus) - loss(minus)) / (2 * eps)
+                scale = max(1.0, float(np.max(np.abs(grad))))
+                assert abs(grad.reshape(-1)[idx] - fd) <= 1e-6 * scale, \
+                    (name, int(idx), float(grad.reshape(-1)[idx]), fd, softplus)
+
+
 MAMBA1_PINS = [pin_closed_form, pin_augmented_matrix, pin_blelloch_order, pin_lti_convolution,
                pin_split_resume, pin_prefix_sum_case, pin_memoryless_case, pin_gate_and_skip,
                pin_softplus_and_bias, pin_decode_steps]
 SSD_PINS = [pin_ssd_is_mamba1, pin_ssd_quadratic, pin_ssd_chunked]
 CONV_PINS = [pin_conv_numpy, pin_conv_one_tap, pin_conv_split_resume, pin_conv_feeds_scan]
-ALL_PINS = MAMBA1_PINS + SSD_PINS + CONV_PINS
+BWD_PINS = [pin_backward_finite_differences]
+ALL_PINS = MAMBA1_PINS + SSD_PINS + CONV_PINS + BWD_PINS

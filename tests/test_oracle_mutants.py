@@ -12,7 +12,7 @@ import subprocess
 import pytest
 
 import oracle
-from oracle_pins import ALL_PINS, CONV_PINS, MAMBA1_PINS, SSD_PINS
+from oracle_pins import ALL_PINS, BWD_PINS, CONV_PINS, MAMBA1_PINS, SSD_PINS
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
 
@@ -20,7 +20,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
 MUTANTS = [
     ("drop_skip", "(j->D ? j->D[d] * u[t] : 0.0)", "0.0", MAMBA1_PINS),
     ("gate_sign", "return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));", ALL_PINS),
-    ("decay_sign", "exp(dt * Ad[n])", "exp(-dt * Ad[n])", MAMBA1_PINS),
+    ("decay_sign", "const double dA = exp(dt * Ad[n]);", "const double dA = exp(-dt * Ad[n]);",
+     MAMBA1_PINS),
     ("input_no_dt", "dt * Bb[n * L + t] * u[t]", "Bb[n * L + t] * u[t]", MAMBA1_PINS),
     ("readout_uses_B", "acc += Cb[n * L + t] * h[n];", "acc += Bb[n * L + t] * h[n];", MAMBA1_PINS),
     ("readout_before_update",
@@ -51,6 +52,15 @@ MUTANTS = [
     ("conv_ignores_window", "else if (j->x_prev)", "else if (0)", CONV_PINS),
     ("conv_time_shift", "const int64_t tt = t - (K - 1) + k;", "const int64_t tt = t - K + k;",
      CONV_PINS),
+    ("bwd_adjoint_not_decayed", "lam[n] *= a;                                      /* carried",
+     "lam[n] *= 1.0;                                    /* carried", BWD_PINS),
+    ("bwd_du_no_dt", "du_t += lam[n] * dt * Bb[n * L + t];", "du_t += lam[n] * Bb[n * L + t];",
+     BWD_PINS),
+    ("bwd_dA_uses_h_t", "if (dA) dA[d * N + n] += lam[n] * dt * a * hp;",
+     "if (dA) dA[d * N + n] += lam[n] * dt * a * hs[(t + 1) * N + n];", BWD_PINS),
+    ("bwd_softplus_grad", "return s > 20.0 ? 1.0 : 1.0 / (1.0 + exp(-s));",
+     "return s > 20.0 ? 1.0 : 1.0 / (1.0 + exp(s));", BWD_PINS),
+    ("bwd_gate_grad", "(sg * (1.0 + zv * (1.0 - sg)))", "(sg * (1.0 + zv * sg))", BWD_PINS),
 ]
 
 
