@@ -465,6 +465,28 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
         "launches_per_call": case.launches}
     del case, cstep
     torch.cuda.empty_cache()
+    # gradients of the scan on the 130M-layer shape (dy fp32, gradients fp32)
+    case = ScanCase(WORKLOAD)
+    t = case.t
+    dy = torch.randn(t["u"].shape, dtype=torch.float32, device="cuda")
+    bws = torch.empty(api.scan_bwd_workspace_size(t["u"], t["delta"], t["A"], t["B"], t["C"],
+                                                  t["D"], t["z"], t["delta_bias"], True),
+                      dtype=torch.uint8, device="cuda")
+    bstep = lambda: api.scan_bwd(t["u"], t["delta"], t["A"], t["B"], t["C"], dy, t["D"], t["z"],
+                                 t["delta_bias"], True, None, workspace=bws)
+    total, per, _ = time_steps(bstep, max(3, steps // 4), warmup, flush, 1, None)
+    sec = total / max(3, steps // 4)
+    c = case.cfg
+    elems = c["batch"] * c["dim"] * c["seqlen"]
+    bc = 2 * c["batch"] * c["dstate"] * c["seqlen"]
+    bbytes = elems * (3 * case.esize + 4 + 3 * 4) + bc * (case.esize + 4)
+    out["mamba130m_layer_bwd"] = {
+        "config": describe(c, True) + ", gradients of every input (fp32)",
+        "us_per_call": round(sec * 1e6, 2), "GB_per_s": round(bbytes / sec / 1e9, 1),
+        "hbm_frac": round(bbytes / sec / 1e9 / hbm_peak, 4),
+        "elems_per_s": round(elems / sec, 1), "launches_per_call": 1}
+    del case, dy, bws, bstep
+    torch.cuda.empty_cache()
     # Mamba-2 chunked scan (tensor cores)
     cfg, sstep, keep = ssd_case()
     total, per, _ = time_steps(sstep, steps, warmup, flush, 1, None)

@@ -173,6 +173,35 @@ ssm_status_t ssm_scan_fwd_varlen(const ssm_scan_args_t* args, const int32_t* cu_
                                  int64_t nseq, void* workspace, size_t workspace_bytes,
                                  ssm_stream_t stream);
 
+/* Gradients of the selective scan (reverse mode) for a loss whose gradient
+ * with respect to y is dy (batch, dim, seqlen) fp32: the states are
+ * recomputed (page "从硬件感知到算法革命" section 1, "recomputation") and the
+ * adjoint lambda[t] = ds_t C[t] + exp(dt'_{t+1} A) lambda[t+1], ds_t = dy_t
+ * silu(z_t), is swept backwards.  `args` as for ssm_scan_fwd (y and h_last
+ * are not used), default contiguous layouts only, one B/C group
+ * (SSM_ERR_UNSUPPORTED otherwise).  Every gradient is fp32, laid out like its
+ * input: du, ddelta, dz (batch, dim, seqlen); dA (dim, dstate); dB, dC
+ * (batch, dstate, seqlen); dD, ddelta_bias (dim); dh0 (batch, dim, dstate).
+ * dA, dB and dC are required; the others may be NULL, and those whose input
+ * is NULL are not written.  Workspace: ssm_scan_bwd_workspace_size bytes
+ * (16-byte aligned) for the state checkpoints. */
+typedef struct {
+  float* du;
+  float* ddelta;
+  float* dz;
+  float* dA;
+  float* dB;
+  float* dC;
+  float* dD;
+  float* ddelta_bias;
+  float* dh0;
+} ssm_scan_grads_t;
+
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_args_t* args);
+ssm_status_t ssm_scan_bwd(const ssm_scan_args_t* args, const float* dy,
+                          const ssm_scan_grads_t* grads, void* workspace, size_t workspace_bytes,
+                          ssm_stream_t stream);
+
 /* Bytes of the library's static device scratch used by ssm_scan_fwd_noalloc. */
 #define SSM_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 

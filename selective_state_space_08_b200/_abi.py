@@ -38,6 +38,11 @@ class ConvArgs(ctypes.Structure):
     _fields_ = [("width", _i64), ("weight", _fp), ("bias", _fp), ("x_prev", _fp)]
 
 
+class ScanGrads(ctypes.Structure):
+    _fields_ = [(k, _fp) for k in ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias",
+                                   "dh0")]
+
+
 class StepArgs(ctypes.Structure):
     _fields_ = [("batch", _i64), ("dim", _i64), ("dstate", _i64), ("dtype", ctypes.c_int),
                 ("u", _vp), ("delta", _vp), ("z", _vp), ("B", _vp), ("C", _vp),
@@ -84,6 +89,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.ssm_scan_fwd_varlen.argtypes = [ctypes.POINTER(ScanArgs), _vp, _i64, _vp, ctypes.c_size_t,
                                         _vp]
     lib.ssm_scan_fwd_varlen.restype = ctypes.c_int
+    lib.ssm_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs)]
+    lib.ssm_scan_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.ssm_scan_bwd.argtypes = [ctypes.POINTER(ScanArgs), _vp, ctypes.POINTER(ScanGrads), _vp,
+                                 ctypes.c_size_t, _vp]
+    lib.ssm_scan_bwd.restype = ctypes.c_int
     lib.ssm_scan_fwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), _vp]
     lib.ssm_scan_fwd_noalloc.restype = ctypes.c_int
     lib.ssm_scan_fwd_host_staging_size.argtypes = [ctypes.POINTER(ScanArgs), _i64]

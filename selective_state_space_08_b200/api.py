@@ -226,6 +226,65 @@ def scan_fwd_varlen(u, delta, A, B, C, cu_seqlens, D=None, z=None, delta_bias=No
     return y, h_last
 
 
+def scan_bwd_workspace_size(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                            delta_softplus=True, h0=None) -> int:
+    """Bytes of scratch ``scan_bwd`` needs for these tensors (state checkpoints)."""
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, None, None)
+    for f in ("u_stride", "delta_stride", "z_stride", "y_stride", "B_stride", "C_stride"):
+        getattr(a, f)[0] = 0
+        getattr(a, f)[1] = 0
+    n = _abi.load().ssm_scan_bwd_workspace_size(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    return int(n)
+
+
+def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softplus=True,
+             h0=None, *, workspace=None, stream=None):
+    """Gradients of the selective scan for a loss with gradient ``dy``
+    (batch, dim, L) float32 with respect to y.  Inputs as for ``scan_fwd``
+    (contiguous).  Returns a dict of float32 tensors: du, ddelta, dA, dB, dC,
+    and dD, dz, ddelta_bias, dh0 for the inputs that are given."""
+    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("dy", dy),
+                    ("D", D), ("z", z), ("delta_bias", delta_bias), ("h0", h0)):
+        _cuda(name, t)
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _cuda("dy", dy, torch.float32)
+    if tuple(dy.shape) != tuple(u.shape):
+        raise ValueError("dy must have the shape of u")
+    a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, None, None)
+    for f in ("u_stride", "delta_stride", "z_stride", "y_stride", "B_stride", "C_stride"):
+        getattr(a, f)[0] = 0
+        getattr(a, f)[1] = 0
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    f32 = lambda *shape: torch.empty(shape, dtype=torch.float32, device=u.device)
+    out = {"du": f32(batch, dim, L), "ddelta": f32(batch, dim, L), "dA": f32(dim, N),
+           "dB": f32(batch, N, L), "dC": f32(batch, N, L)}
+    if D is not None:
+        out["dD"] = f32(dim)
+    if z is not None:
+        out["dz"] = f32(batch, dim, L)
+    if delta_bias is not None:
+        out["ddelta_bias"] = f32(dim)
+    if h0 is not None:
+        out["dh0"] = f32(batch, dim, N)
+    g = _abi.ScanGrads()
+    for k in ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dh0"):
+        setattr(g, k, _ptr(out.get(k)))
+    lib = _abi.load()
+    need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid arguments")
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(int(need), dtype=torch.uint8, device=u.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _abi.check(lib.ssm_scan_bwd(ctypes.byref(a), _ptr(dy), ctypes.byref(g), _ptr(workspace),
+                                ws_bytes, _stream(stream)), "ssm_scan_bwd")
+    return out
+
+
 def scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
                      h0=None, *, y, h_last=None, stream=None):
     """``scan_fwd`` for callers that cannot allocate device memory: ``y`` (and

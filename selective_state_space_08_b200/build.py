@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libssmscan.so")
 SOURCES = ["api.cu"]
-HEADERS = ["common.cuh", "exp2_poly.cuh", "scan_fwd.cuh", "scan_step.cuh", "ssd_fwd.cuh", "tc.cuh"]
+HEADERS = ["common.cuh", "exp2_poly.cuh", "scan_fwd.cuh", "scan_bwd.cuh", "scan_step.cuh", "ssd_fwd.cuh", "tc.cuh"]
 
 
 def nvcc() -> str:

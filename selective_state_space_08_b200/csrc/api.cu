@@ -13,6 +13,7 @@
 #include <utility>
 
 #include "../../include/ssmscan.h"
+#include "scan_bwd.cuh"
 #include "scan_fwd.cuh"
 #include "scan_step.cuh"
 #include "ssd_fwd.cuh"
@@ -659,9 +660,114 @@ ssm_status_t scan_fwd_impl(const ssm_scan_args_t* args, const ssm_conv_args_t* c
   return plan.vec ? run_fwd<float, true, false>(p, stream) : run_fwd<float, false, false>(p, stream);
 }
 
+// ---- gradients -------------------------------------------------------------------------
+ssm_status_t plan_bwd(const ssm_scan_args_t* a, BwdParams* p, size_t* ws_bytes, bool check_ptrs) {
+  ScanPlan plan;
+  ssm_status_t st = plan_scan(a, &plan, false);  // y and h_last play no part here
+  if (st != SSM_OK) return st;
+  if (check_ptrs && a->batch > 0 && a->dim > 0) {
+    if (a->A == nullptr) return SSM_ERR_INVALID_ARG;
+    if (a->seqlen > 0 && (a->u == nullptr || a->delta == nullptr || a->B == nullptr ||
+                          a->C == nullptr))
+      return SSM_ERR_INVALID_ARG;
+  }
+  const int64_t* strides[] = {a->u_stride, a->delta_stride, a->z_stride,
+                              a->y_stride, a->B_stride, a->C_stride};
+  for (const int64_t* s : strides)
+    if (s[0] != 0 || s[1] != 0) return SSM_ERR_UNSUPPORTED;
+  if (a->ngroups > 1) return SSM_ERR_UNSUPPORTED;
+  p->batch = a->batch;
+  p->dim = a->dim;
+  p->dstate = a->dstate;
+  p->seqlen = a->seqlen;
+  p->u = a->u;
+  p->delta = a->delta;
+  p->z = a->z;
+  p->B = a->B;
+  p->C = a->C;
+  p->A = a->A;
+  p->D = a->D;
+  p->bias = a->delta_bias;
+  p->softplus = a->delta_softplus ? 1 : 0;
+  p->h0 = a->h0;
+  p->nblk = (a->seqlen + bwd::kBlk - 1) / bwd::kBlk;
+  p->nchb = (a->dim + bwd::kCh - 1) / bwd::kCh;
+  const size_t ckpt = static_cast<size_t>(a->batch) * a->dim * bwd::kStates * p->nblk;
+  const size_t part = 2 * static_cast<size_t>(p->nchb) * a->batch * a->dstate * a->seqlen;
+  *ws_bytes = (ckpt + part) * sizeof(float);
+  return SSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_args_t* args) {
+  BwdParams p;
+  size_t ws = 0;
+  if (plan_bwd(args, &p, &ws, false) != SSM_OK) return static_cast<size_t>(-1);
+  return ws;
+}
+
+ssm_status_t ssm_scan_bwd(const ssm_scan_args_t* args, const float* dy, const ssm_scan_grads_t* g,
+                          void* workspace, size_t workspace_bytes, ssm_stream_t stream_) {
+  if (g == nullptr) return SSM_ERR_INVALID_ARG;
+  BwdParams p;
+  size_t ws = 0;
+  ssm_status_t st = plan_bwd(args, &p, &ws, true);
+  if (st != SSM_OK) return st;
+  if (p.batch == 0 || p.dim == 0) return SSM_OK;
+  if (dy == nullptr && p.seqlen > 0) return SSM_ERR_INVALID_ARG;
+  if (g->dA == nullptr || g->dB == nullptr || g->dC == nullptr) return SSM_ERR_INVALID_ARG;
+  const void* f32s[] = {dy, g->du, g->ddelta, g->dz, g->dA, g->dB, g->dC, g->dD, g->ddelta_bias,
+                        g->dh0};
+  for (const void* t : f32s)
+    if (t != nullptr && !aligned(t, 4)) return SSM_ERR_ALIGNMENT;
+  if (ws > 0 && (workspace == nullptr || workspace_bytes < ws)) return SSM_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return SSM_ERR_ALIGNMENT;
+  p.dy = dy;
+  p.du = g->du;
+  p.ddelta = g->ddelta;
+  p.dz = args->z ? g->dz : nullptr;
+  p.dA = g->dA;
+  p.dB = g->dB;
+  p.dC = g->dC;
+  p.dD = args->D ? g->dD : nullptr;
+  p.dbias = args->delta_bias ? g->ddelta_bias : nullptr;
+  p.dh0 = args->h0 ? g->dh0 : nullptr;
+  p.ckpt = static_cast<float*>(workspace);
+  p.part = p.ckpt + static_cast<size_t>(p.batch) * p.dim * bwd::kStates * p.nblk;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  // the accumulated gradients start from zero (dB and dC are written whole)
+  const size_t bnl = static_cast<size_t>(p.batch) * p.dstate * p.seqlen;
+  st = cuda_status(cudaMemsetAsync(p.dA, 0, static_cast<size_t>(p.dim) * p.dstate * sizeof(float),
+                                   stream), "scan_bwd: zero dA");
+  if (st == SSM_OK && p.dD)
+    st = cuda_status(cudaMemsetAsync(p.dD, 0, p.dim * sizeof(float), stream), "scan_bwd: zero dD");
+  if (st == SSM_OK && p.dbias)
+    st = cuda_status(cudaMemsetAsync(p.dbias, 0, p.dim * sizeof(float), stream),
+                     "scan_bwd: zero bias gradient");
+  if (st != SSM_OK) return st;
+  const dim3 grid(static_cast<unsigned>((p.dim + bwd::kCh - 1) / bwd::kCh),
+                  static_cast<unsigned>(p.batch));
+  const size_t smem = sizeof(bwd::Smem);
+  if (args->dtype == SSM_BF16) {
+    auto kernel = bwd::scan_bwd_kernel<__nv_bfloat16>;
+    st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem), "scan_bwd: opt-in");
+    if (st != SSM_OK) return st;
+    kernel<<<grid, bwd::kThreads, smem, stream>>>(p);
+  } else {
+    auto kernel = bwd::scan_bwd_kernel<float>;
+    st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem), "scan_bwd: opt-in");
+    if (st != SSM_OK) return st;
+    kernel<<<grid, bwd::kThreads, smem, stream>>>(p);
+  }
+  st = cuda_status(cudaGetLastError(), "scan_bwd: launch");
+  if (st != SSM_OK || bnl == 0) return st;
+  bwd::scan_bwd_reduce_bc<<<static_cast<unsigned>((bnl + 255) / 256), 256, 0, stream>>>(p);
+  return cuda_status(cudaGetLastError(), "scan_bwd: dB / dC reduction launch");
+}
+
 
 size_t ssm_scan_fwd_workspace_size(const ssm_scan_args_t* args) {
   ScanPlan plan;

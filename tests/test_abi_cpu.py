@@ -131,6 +131,25 @@ def test_varlen_scan_host_checks(lib):
     assert lib.ssm_scan_fwd_varlen(ctypes.byref(a), 0x10002, 2, None, 0, None) == 3
 
 
+def test_backward_host_checks(lib):
+    a = _args(batch=2, dim=40, seqlen=100)
+    need = lib.ssm_scan_bwd_workspace_size(ctypes.byref(a))
+    # checkpoints (16 states x ceil(100 / 16) blocks) and per-channel-block dB / dC partials
+    assert need == (2 * 40 * 16 * 7 + 2 * 2 * 2 * 16 * 100) * 4
+    g = _abi.ScanGrads()
+    assert lib.ssm_scan_bwd(ctypes.byref(a), 0x10000, None, None, 0, None) == 1
+    assert lib.ssm_scan_bwd(ctypes.byref(a), 0x10000, ctypes.byref(g), None, 0, None) == 1
+    g.dA, g.dB, g.dC = 0x10000, 0x10000, 0x10000
+    assert lib.ssm_scan_bwd(ctypes.byref(a), 0x10000, ctypes.byref(g), None, 0, None) == 5
+    a.y = None  # the forward output plays no part in the gradients
+    assert lib.ssm_scan_bwd(ctypes.byref(a), 0x10000, ctypes.byref(g), None, 0, None) == 5
+    a.u = None
+    assert lib.ssm_scan_bwd(ctypes.byref(a), 0x10000, ctypes.byref(g), None, 0, None) == 1
+    s = _args(batch=2, dim=40, seqlen=100)
+    s.u_stride[1] = 128
+    assert lib.ssm_scan_bwd_workspace_size(ctypes.byref(s)) == ctypes.c_size_t(-1).value
+
+
 def test_conv_scan_rejects_bad_stage_arguments(lib):
     a = _args()
     c = _abi.ConvArgs()
