@@ -30,9 +30,11 @@
  * and returns the final state h_L.  The skip term sits inside the gate.
  *
  * Conventions shared by every entry point:
- *  - All tensor pointers are DEVICE pointers owned by the caller.  The
- *    library allocates no device memory; scratch is passed as `workspace`
- *    of the size the matching *_workspace_size call reports.
+ *  - All tensor pointers are DEVICE pointers owned by the caller, except
+ *    those of ssm_scan_fwd_host, which are host pointers.  The library
+ *    allocates no device memory; scratch is passed as `workspace` (or
+ *    `staging`) of the size the matching *_size call reports, or, for
+ *    ssm_scan_fwd_noalloc, comes from a static array.
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).
  *    Argument checks run on the host before any launch and return
  *    synchronously; a failed launch returns SSM_ERR_CUDA.
