@@ -750,13 +750,14 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_args_t* args, const float* dy, const ss
   if (st != SSM_OK) return st;
   const dim3 grid(static_cast<unsigned>((p.dim + bwd::kCh - 1) / bwd::kCh),
                   static_cast<unsigned>(p.batch));
-  const size_t smem = sizeof(bwd::Smem);
   if (args->dtype == SSM_BF16) {
+    const size_t smem = sizeof(bwd::Smem<__nv_bfloat16>);
     auto kernel = bwd::scan_bwd_kernel<__nv_bfloat16>;
     st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem), "scan_bwd: opt-in");
     if (st != SSM_OK) return st;
     kernel<<<grid, bwd::kThreads, smem, stream>>>(p);
   } else {
+    const size_t smem = sizeof(bwd::Smem<float>);
     auto kernel = bwd::scan_bwd_kernel<float>;
     st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem), "scan_bwd: opt-in");
     if (st != SSM_OK) return st;
