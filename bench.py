@@ -42,7 +42,7 @@ METRIC = "selective_scan_fwd HBM GB/s (% of B200 peak) and B·D·L elems/s"
 L2_FLUSH_BYTES = 512 << 20   # written between timed steps (L2 is 126 MB)
 SM_COUNT_NOMINAL = 148
 SM_MAX_MHZ_NOMINAL = 1965.0
-FP32_LANES_PER_SM = 128      # measured on this machine: 127.9 lane-ops/SM/clk
+FP32_LANES_PER_SM = 128      # measured on B200: 127.9 lane-ops/SM/clk
 MUFU_LANES_PER_SM = 16       # measured: 16.0 ex2 / lg2 / tanh per SM per clk
 EXP_POLY_LANE_OPS = 8        # FMA-pipe cost of one range-reduced degree-5 exp2
 
