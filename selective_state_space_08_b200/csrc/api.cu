@@ -181,7 +181,7 @@ ssm_status_t plan_scan(const ssm_scan_args_t* a, ScanPlan* out, bool check_ptrs 
 template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV, bool VARLEN>
 ssm_status_t launch_fwd(const ScanParams& p, cudaStream_t stream) {
   auto kernel = fwd::scan_fwd_kernel<T, MODE, HAS_Z, VEC, CONV, VARLEN>;
-  const size_t smem = sizeof(fwd::Smem<T, CONV>);
+  const size_t smem = sizeof(fwd::Smem<T, CONV, fwd::packed_bc<T, MODE, HAS_Z>()>);
   ssm_status_t st = cuda_status(set_smem(reinterpret_cast<const void*>(kernel), smem),
                                 "scan_fwd: shared-memory opt-in");
   if (st != SSM_OK) return st;

@@ -23,10 +23,11 @@
 // Data movement.  Each input element is read from HBM once: tiles of kTL time
 // steps of u and delta (kCH rows) and of B and C (16 rows) are staged into
 // shared memory with 16-byte cp.async copies; the next tile's copies are in
-// flight during the current tile's scan.  Per tile the block converts B and
-// C to fp32 once (shared by every channel of the batch) and computes dt'
-// (clamped for the decay argument) and dt' u once per element (shared by the
-// 4 lanes of a channel).  The partial sums C.h of the 4 lanes are reduced
+// flight during the current tile's scan.  Per tile the block transposes B
+// and C once into [step][state] rows (shared by every channel of the batch;
+// bf16 inputs stay bf16 there, fp32 inputs fp32) and computes dt' (clamped
+// for the decay argument) and dt' u once per element (shared by the 4 lanes
+// of a channel).  The partial sums C.h of the 4 lanes are reduced
 // with a shuffle butterfly per 8-step sub-tile; each lane then finishes 2 steps
 // (skip term, gate, rounding), reading z and writing y straight from and to
 // global memory.
@@ -41,6 +42,8 @@
 // exp(A sum_t dt'_t); the full pass (MODE kFull) then runs every segment from
 // its incoming state.  No block ever waits on another.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 #include "exp2_poly.cuh"
 
@@ -93,11 +96,37 @@ constexpr int kFull = 0, kAgg = 1;
 // |dt' A log2(e)| is clamped to this before the decay exponential: beyond it
 // the decay is below 2^-126 (or the state overflows anyway).
 constexpr float kMaxDecayArg = 126.0f;
-// fp32 B / C rows of 20 floats: the prep's stores of 8 consecutive steps from
-// one quarter-warp then land in 8 distinct 4-bank groups.
+// B / C rows of 20 words: the prep's 16-byte stores of 8 consecutive steps
+// from one quarter-warp then land in 8 distinct 4-bank groups.
 constexpr int kBCRow = kMaxN + 4;
 
-template <typename T, bool CONV = false>
+// B and C of each step in [step][state] rows, in the form the recurrence reads.
+// fp32 rows: separate B and C rows, lane g reads words 4g .. 4g+3 of each.
+template <bool PACKED>
+struct alignas(16) BCRows {
+  float B[kTL][kBCRow];
+  float C[kTL][kBCRow];
+};
+// Packed rows (bf16 inputs, kept bf16: widening to fp32 is exact): words 4g,
+// 4g+1 of a row hold the bf16 pairs B(4g, 4g+1), B(4g+2, 4g+3) and words
+// 4g+2, 4g+3 the same states of C, so one 16-byte shared load gives lane g
+// both operands of a step, half the shared-memory wavefronts of fp32 rows.
+template <>
+struct alignas(16) BCRows<true> {
+  uint32_t w[kTL][kBCRow];
+};
+
+// Which rows a variant reads.  Widening packed rows costs 8 integer operations
+// per lane and step: that pays where the shared-memory pipe limits (variants
+// without the gate, 5 blocks per SM; 588 against 620 us on a 4 x 5120 x 4096
+// scan) but not in the gated full pass, whose warps at 3 blocks per SM wait
+// on latency (215 against 207 us on an 8 x 1536 x 2048 scan).
+template <typename T, int MODE, bool HAS_Z>
+constexpr bool packed_bc() {
+  return std::is_same_v<T, __nv_bfloat16> && !(HAS_Z && MODE == kFull);
+}
+
+template <typename T, bool CONV = false, bool PACKED = false>
 struct Smem {
   static constexpr int kEPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
   // A raw row holds a tile plus a 16-byte pad, so consecutive rows start 4
@@ -110,8 +139,7 @@ struct Smem {
   T raw_C[kMaxN][kRow];
   float dtp[kCH][kTL + 4];   // dt', clamped, per (channel, step): decay argument
   float du[kCH][kTL + 4];    // dt' * u
-  float Bf[kTL][kBCRow];     // fp32 B, [step][state]
-  float Cf[kTL][kBCRow];
+  BCRows<PACKED> bc;         // B, C of the tile, [step][state]
   // convolution output u (fp32) for the epilogue's skip term; rows of 72
   // floats put the epilogue's 8-byte reads on distinct banks
   float uc[CONV ? kCH : 1][kTL + 8];
@@ -238,6 +266,74 @@ __device__ __forceinline__ void copy_rows_scalar(T* dst, const T* base, int64_t 
   }
 }
 
+// Two bf16 values packed in a word (low half first) widened to fp32.
+__device__ __forceinline__ float2 widen_pair(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// The tile prep's B / C rows for the steps t of thread (t % 32, q = thread / 32):
+// states 4q .. 4q+3 of step t, from the staged [state][step] rows.
+template <typename T, bool PACKED, bool WITH_C>
+__device__ __forceinline__ void store_bc(BCRows<PACKED>& bc, const T (*raw_B)[Smem<T>::kRow],
+                                         const T (*raw_C)[Smem<T>::kRow], int t, int q) {
+  if constexpr (PACKED) {
+    static_assert(std::is_same_v<T, __nv_bfloat16>, "packed rows hold bf16");
+    auto pack = [&](const T (*raw)[Smem<T>::kRow], int n) {
+      return static_cast<uint32_t>(__bfloat16_as_ushort(raw[n][t])) |
+             (static_cast<uint32_t>(__bfloat16_as_ushort(raw[n + 1][t])) << 16);
+    };
+    const uint32_t b0 = pack(raw_B, 4 * q), b1 = pack(raw_B, 4 * q + 2);
+    if (WITH_C) {
+      *reinterpret_cast<uint4*>(&bc.w[t][4 * q]) =
+          make_uint4(b0, b1, pack(raw_C, 4 * q), pack(raw_C, 4 * q + 2));
+    } else {
+      *reinterpret_cast<uint2*>(&bc.w[t][4 * q]) = make_uint2(b0, b1);
+    }
+  } else {
+    *reinterpret_cast<float4*>(&bc.B[t][4 * q]) =
+        make_float4(to_f32<T>(raw_B[4 * q + 0][t]), to_f32<T>(raw_B[4 * q + 1][t]),
+                    to_f32<T>(raw_B[4 * q + 2][t]), to_f32<T>(raw_B[4 * q + 3][t]));
+    if (WITH_C)
+      *reinterpret_cast<float4*>(&bc.C[t][4 * q]) =
+          make_float4(to_f32<T>(raw_C[4 * q + 0][t]), to_f32<T>(raw_C[4 * q + 1][t]),
+                      to_f32<T>(raw_C[4 * q + 2][t]), to_f32<T>(raw_C[4 * q + 3][t]));
+  }
+}
+
+// B of step t for lane g's state pairs (4g, 4g+1), (4g+2, 4g+3); from packed
+// rows with WITH_C also C, which comes in the same 16-byte load.
+template <bool PACKED, bool WITH_C>
+__device__ __forceinline__ void load_b(const BCRows<PACKED>& bc, int t, int g, float2& b01,
+                                       float2& b23, float2& c01, float2& c23) {
+  if constexpr (PACKED) {
+    if (WITH_C) {
+      const uint4 w = *reinterpret_cast<const uint4*>(&bc.w[t][4 * g]);
+      b01 = widen_pair(w.x);
+      b23 = widen_pair(w.y);
+      c01 = widen_pair(w.z);
+      c23 = widen_pair(w.w);
+    } else {
+      const uint2 w = *reinterpret_cast<const uint2*>(&bc.w[t][4 * g]);
+      b01 = widen_pair(w.x);
+      b23 = widen_pair(w.y);
+    }
+  } else {
+    const float4 bq = *reinterpret_cast<const float4*>(&bc.B[t][4 * g]);
+    b01 = make_float2(bq.x, bq.y);
+    b23 = make_float2(bq.z, bq.w);
+  }
+}
+// C of step t from fp32 rows, read where it is used (packed rows gave it with B).
+template <bool PACKED>
+__device__ __forceinline__ void load_c(const BCRows<PACKED>& bc, int t, int g, float2& c01,
+                                       float2& c23) {
+  if constexpr (!PACKED) {
+    const float4 cq = *reinterpret_cast<const float4*>(&bc.C[t][4 * g]);
+    c01 = make_float2(cq.x, cq.y);
+    c23 = make_float2(cq.z, cq.w);
+  }
+}
+
 // Two consecutive elements kept in their storage format until used.
 template <typename T>
 struct RawPair;
@@ -288,10 +384,26 @@ __device__ __forceinline__ void sub_decays(const float* dtp_row, float2 A01, flo
   }
 }
 
+// Blocks per SM that the register budget of a packed-row variant must allow:
+// what its shared memory allows (5, 4 with the convolution output rows), or
+// 3 for packed batches, whose state needs about 160 registers.  Without this
+// the compiler gives the packed no-gate pass 128 registers (4 blocks).  The
+// fp32-row variants keep the compiler's own allocation (0: no minimum).
+template <typename T, int MODE, bool HAS_Z, bool CONV, bool VARLEN>
+constexpr int min_blocks() {
+  if (!packed_bc<T, MODE, HAS_Z>()) return 0;
+  if (MODE == kAgg) return 5;
+  if (VARLEN) return 3;
+  if (CONV) return 4;
+  return 5;
+}
+
 template <typename T, int MODE, bool HAS_Z, bool VEC, bool CONV = false, bool VARLEN = false>
-__global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) {
+__global__ void __launch_bounds__(kThreads, (min_blocks<T, MODE, HAS_Z, CONV, VARLEN>()))
+    scan_fwd_kernel(const ScanParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  Smem<T, CONV>& sm = *reinterpret_cast<Smem<T, CONV>*>(smem_raw);
+  constexpr bool kPacked = packed_bc<T, MODE, HAS_Z>();
+  Smem<T, CONV, kPacked>& sm = *reinterpret_cast<Smem<T, CONV, kPacked>*>(smem_raw);
   constexpr bool kGate = HAS_Z && MODE == kFull;
 
   const int tid = threadIdx.x;
@@ -444,21 +556,13 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
       sm.vl_end = en;
       sm.vl_seq = lo;
     }
-    {  // B and C to fp32, [step][state]: thread -> states 4q .. 4q+3, steps r and r + 32
+    {  // B and C to [step][state] rows: thread -> states 4q .. 4q+3, steps r and r + 32
       static_assert(kThreads == 128 && kTL == 64 && kMaxN == 16, "prep mapping");
       const int r = tid % 32;
       const int q = tid / 32;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int t = r + 32 * h;
-        *reinterpret_cast<float4*>(&sm.Bf[t][4 * q]) =
-            make_float4(to_f32<T>(sm.raw_B[4 * q + 0][t]), to_f32<T>(sm.raw_B[4 * q + 1][t]),
-                        to_f32<T>(sm.raw_B[4 * q + 2][t]), to_f32<T>(sm.raw_B[4 * q + 3][t]));
-        if (MODE == kFull)
-          *reinterpret_cast<float4*>(&sm.Cf[t][4 * q]) =
-              make_float4(to_f32<T>(sm.raw_C[4 * q + 0][t]), to_f32<T>(sm.raw_C[4 * q + 1][t]),
-                          to_f32<T>(sm.raw_C[4 * q + 2][t]), to_f32<T>(sm.raw_C[4 * q + 3][t]));
-      }
+      for (int h = 0; h < 2; ++h)
+        store_bc<T, kPacked, MODE == kFull>(sm.bc, sm.raw_B, sm.raw_C, r + 32 * h, q);
     }
     {  // dt' and dt' u of channel pc, steps [pt0, pt0 + 16)
       // the convolution's window: three inputs before pt0 (the previous
@@ -529,8 +633,6 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
       for (int s = 0; s < kTL / kSub; ++s) zt[s] = zn[s];
       if (k + 1 < ntiles) prefetch_z(zn, t0 + kTL);
     }
-    const float* bf = &sm.Bf[0][kNPT * g];
-    const float* cf = &sm.Cf[0][kNPT * g];
     const unsigned long long vstart = VARLEN ? sm.vl_start : 0ull;
     const unsigned long long vend = VARLEN ? sm.vl_end : 0ull;
     if (VARLEN && vstart != 0ull) restarted = true;
@@ -554,12 +656,13 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
 #pragma unroll
       for (int tt = 0; tt < kSub; ++tt) {
         const int t = tb + tt;
-        const float4 bq = *reinterpret_cast<const float4*>(bf + t * kBCRow);
+        float2 b01, b23, c01, c23;
+        load_b<kPacked, MODE == kFull>(sm.bc, t, g, b01, b23, c01, c23);
         const float2 du2 = make_float2(dus[tt], dus[tt]);
         float2 a01 = dcur.a01[tt], a23 = dcur.a23[tt];
         if (VARLEN && ((vstart >> t) & 1ull)) a01 = a23 = make_float2(0.f, 0.f);  // restart
-        h01 = __ffma2_rn(a01, h01, __fmul2_rn(du2, make_float2(bq.x, bq.y)));
-        h23 = __ffma2_rn(a23, h23, __fmul2_rn(du2, make_float2(bq.z, bq.w)));
+        h01 = __ffma2_rn(a01, h01, __fmul2_rn(du2, b01));
+        h23 = __ffma2_rn(a23, h23, __fmul2_rn(du2, b23));
         if (VARLEN && MODE == kFull && ((vend >> t) & 1ull) && ch_ok && p.h_last != nullptr) {
           // the last step of a sequence: its state goes to h_last[sequence]
           const unsigned long long upto = t == 63 ? ~0ull : ((2ull << t) - 1ull);
@@ -573,9 +676,9 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(const ScanParams p) 
           }
         }
         if (MODE == kFull) {
-          const float4 cq = *reinterpret_cast<const float4*>(cf + t * kBCRow);
-          float2 yv = __fmul2_rn(make_float2(cq.x, cq.y), h01);
-          yv = __ffma2_rn(make_float2(cq.z, cq.w), h23, yv);
+          load_c<kPacked>(sm.bc, t, g, c01, c23);
+          float2 yv = __fmul2_rn(c01, h01);
+          yv = __ffma2_rn(c23, h23, yv);
           ys[tt] = yv.x + yv.y;
         }
       }
