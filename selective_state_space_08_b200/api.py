@@ -20,8 +20,26 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _one_device(named):
+    """The CUDA device of the given tensors, which must all be on it (the
+    library reads every operand on the device it launches on)."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other tensors on {dev}")
+    return dev
+
+
+def _stream(stream, device):
+    """The stream to launch on: ``stream``, which must belong to ``device``,
+    or the current torch stream of ``device``."""
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    if s.device != device:
+        raise ValueError(f"stream is on {s.device}, the tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -121,9 +139,12 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     u, delta, z: (batch, dim, L) float32 or bfloat16, unit stride along L;
     B, C: (batch, N, L) same dtype; A: (dim, N) float32; D, delta_bias: (dim,)
     float32; h0: (batch, dim, N) float32.  Returns (y, h_last)."""
-    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
-                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+    named = (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+             ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last),
+             ("workspace", workspace))
+    for name, t in named:
         _cuda(name, t)
+    dev = _one_device(named)
     if u.dim() != 3:
         raise ValueError("u must be (batch, dim, L)")
     if y is None:
@@ -139,8 +160,9 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(int(need), dtype=torch.uint8, device=u.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _abi.check(lib.ssm_scan_fwd(ctypes.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
-               "ssm_scan_fwd")
+    with torch.cuda.device(dev):
+        _abi.check(lib.ssm_scan_fwd(ctypes.byref(a), _ptr(workspace), ws_bytes,
+                                    _stream(stream, dev)), "ssm_scan_fwd")
     return y, h_last
 
 
@@ -153,9 +175,13 @@ def scan_fwd_conv(x, conv_weight, conv_bias, x_prev, delta, A, B, C, D=None, z=N
     width) float32, width 1..4; conv_bias: (dim,) float32 or None; x_prev:
     (batch, dim, width - 1) float32 or None (inputs before step 0).
     Returns (y, h_last)."""
-    for name, t in (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
-                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+    named = (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+             ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last),
+             ("conv_weight", conv_weight), ("conv_bias", conv_bias), ("x_prev", x_prev),
+             ("workspace", workspace))
+    for name, t in named:
         _cuda(name, t)
+    dev = _one_device(named)
     if x.dim() != 3:
         raise ValueError("x must be (batch, dim, L)")
     batch, dim, _ = x.shape
@@ -183,8 +209,9 @@ def scan_fwd_conv(x, conv_weight, conv_bias, x_prev, delta, A, B, C, D=None, z=N
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(int(need), dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _abi.check(lib.ssm_scan_fwd_conv(ctypes.byref(a), ctypes.byref(c), _ptr(workspace), ws_bytes,
-                                     _stream(stream)), "ssm_scan_fwd_conv")
+    with torch.cuda.device(dev):
+        _abi.check(lib.ssm_scan_fwd_conv(ctypes.byref(a), ctypes.byref(c), _ptr(workspace),
+                                         ws_bytes, _stream(stream, dev)), "ssm_scan_fwd_conv")
     return y, h_last
 
 
@@ -195,10 +222,13 @@ def scan_fwd_varlen(u, delta, A, B, C, cu_seqlens, D=None, z=None, delta_bias=No
     (1, dim, L) and B, C (1, N, L) (or grouped), holding the sequences end to
     end; cu_seqlens: int32 CUDA tensor (nseq + 1) of sequence offsets.  Each
     sequence starts from a zero state.  Returns (y, h_last (nseq, dim, N))."""
-    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
-                    ("delta_bias", delta_bias), ("y", y), ("h_last", h_last)):
+    named = (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+             ("delta_bias", delta_bias), ("y", y), ("h_last", h_last), ("cu_seqlens", cu_seqlens),
+             ("workspace", workspace))
+    for name, t in named:
         _cuda(name, t)
     _cuda("cu_seqlens", cu_seqlens, torch.int32, 1)
+    dev = _one_device(named)
     if not cu_seqlens.is_contiguous() or cu_seqlens.numel() < 2:
         raise ValueError("cu_seqlens must be a contiguous int32 vector of nseq + 1 offsets")
     if u.dim() != 3 or u.shape[0] != 1:
@@ -221,8 +251,10 @@ def scan_fwd_varlen(u, delta, A, B, C, cu_seqlens, D=None, z=None, delta_bias=No
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(int(need), dtype=torch.uint8, device=u.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _abi.check(lib.ssm_scan_fwd_varlen(ctypes.byref(a), _ptr(cu_seqlens), nseq, _ptr(workspace),
-                                       ws_bytes, _stream(stream)), "ssm_scan_fwd_varlen")
+    with torch.cuda.device(dev):
+        _abi.check(lib.ssm_scan_fwd_varlen(ctypes.byref(a), _ptr(cu_seqlens), nseq,
+                                           _ptr(workspace), ws_bytes, _stream(stream, dev)),
+                   "ssm_scan_fwd_varlen")
     return y, h_last
 
 
@@ -245,12 +277,15 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softp
     (batch, dim, L) float32 with respect to y.  Inputs as for ``scan_fwd``
     (contiguous).  Returns a dict of float32 tensors: du, ddelta, dA, dB, dC,
     and dD, dz, ddelta_bias, dh0 for the inputs that are given."""
-    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("dy", dy),
-                    ("D", D), ("z", z), ("delta_bias", delta_bias), ("h0", h0)):
+    named = (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("dy", dy), ("D", D),
+             ("z", z), ("delta_bias", delta_bias), ("h0", h0))
+    for name, t in named:
         _cuda(name, t)
         if t is not None and not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
     _cuda("dy", dy, torch.float32)
+    _cuda("workspace", workspace)
+    dev = _one_device(named + (("workspace", workspace),))
     if tuple(dy.shape) != tuple(u.shape):
         raise ValueError("dy must have the shape of u")
     a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, None, None)
@@ -280,8 +315,9 @@ def scan_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, delta_softp
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(int(need), dtype=torch.uint8, device=u.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _abi.check(lib.ssm_scan_bwd(ctypes.byref(a), _ptr(dy), ctypes.byref(g), _ptr(workspace),
-                                ws_bytes, _stream(stream)), "ssm_scan_bwd")
+    with torch.cuda.device(dev):
+        _abi.check(lib.ssm_scan_bwd(ctypes.byref(a), _ptr(dy), ctypes.byref(g), _ptr(workspace),
+                                    ws_bytes, _stream(stream, dev)), "ssm_scan_bwd")
     return out
 
 
@@ -292,12 +328,15 @@ def scan_fwd_noalloc(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_s
     library's static 4 MiB device array (see ssm_scan_fwd_noalloc in
     include/ssmscan.h: first call on a device before any stream capture;
     overlapping calls race on the shared array)."""
-    for name, t in (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
-                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+    named = (("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+             ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last))
+    for name, t in named:
         _cuda(name, t)
+    dev = _one_device(named)
     a = _scan_args(u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, y, h_last)
-    _abi.check(_abi.load().ssm_scan_fwd_noalloc(ctypes.byref(a), _stream(stream)),
-               "ssm_scan_fwd_noalloc")
+    with torch.cuda.device(dev):
+        _abi.check(_abi.load().ssm_scan_fwd_noalloc(ctypes.byref(a), _stream(stream, dev)),
+                   "ssm_scan_fwd_noalloc")
     return y, h_last
 
 
@@ -343,14 +382,16 @@ def scan_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_soft
     need = lib.ssm_scan_fwd_host_staging_size(ctypes.byref(a), int(slice_batch))
     if need == ctypes.c_size_t(-1).value:
         raise ValueError("invalid arguments")
-    if staging is None or staging.numel() * staging.element_size() < need:
-        staging = torch.empty(max(int(need), 1), dtype=torch.uint8, device="cuda")
     _cuda("staging", staging)
-    s = stream if stream is not None else torch.cuda.current_stream()
-    _abi.check(lib.ssm_scan_fwd_host(ctypes.byref(a), int(slice_batch), _ptr(staging),
-                                     staging.numel() * staging.element_size(),
-                                     ctypes.c_void_p(s.cuda_stream)),
-               "ssm_scan_fwd_host")
+    dev = staging.device if staging is not None else (
+        stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device()))
+    if staging is None or staging.numel() * staging.element_size() < need:
+        staging = torch.empty(max(int(need), 1), dtype=torch.uint8, device=dev)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    with torch.cuda.device(dev):
+        _abi.check(lib.ssm_scan_fwd_host(ctypes.byref(a), int(slice_batch), _ptr(staging),
+                                         staging.numel() * staging.element_size(),
+                                         _stream(s, dev)), "ssm_scan_fwd_host")
     if synchronize:
         s.synchronize()
     return y, h_last
@@ -360,11 +401,13 @@ def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_s
               *, y=None, stream=None):
     """One decode step; ``state`` (batch, dim, N) float32 is updated in place.
     u, delta, z: (batch, dim); B, C: (batch, N).  Returns y (batch, dim)."""
-    for name, t in (("state", state), ("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C),
-                    ("D", D), ("z", z), ("delta_bias", delta_bias), ("y", y)):
+    named = (("state", state), ("u", u), ("delta", delta), ("A", A), ("B", B), ("C", C),
+             ("D", D), ("z", z), ("delta_bias", delta_bias), ("y", y))
+    for name, t in named:
         _cuda(name, t)
         if t is not None and not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    dev = _one_device(named)
     if u.dtype not in _DT:
         raise ValueError("u must be float32 or bfloat16")
     batch, dim = u.shape
@@ -386,7 +429,9 @@ def scan_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_s
     a.A, a.D, a.delta_bias = _ptr(A), _ptr(D), _ptr(delta_bias)
     a.delta_softplus = 1 if delta_softplus else 0
     a.state, a.y = _ptr(state), _ptr(y)
-    _abi.check(_abi.load().ssm_scan_step(ctypes.byref(a), _stream(stream)), "ssm_scan_step")
+    with torch.cuda.device(dev):
+        _abi.check(_abi.load().ssm_scan_step(ctypes.byref(a), _stream(stream, dev)),
+                   "ssm_scan_step")
     return y
 
 
@@ -410,11 +455,14 @@ def ssd_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=T
     (batch, L, N) bfloat16; A, D, delta_bias: (H,) float32; h0: (batch, H, P, N)
     float32.  Returns (y, h_last).  With ``check_status`` the call waits for the
     GPU and raises if a tensor-core wait inside the kernels gave up."""
-    for name, t in (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
-                    ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last)):
+    named = (("x", x), ("delta", delta), ("A", A), ("B", B), ("C", C), ("D", D), ("z", z),
+             ("delta_bias", delta_bias), ("h0", h0), ("y", y), ("h_last", h_last))
+    for name, t in named:
         _cuda(name, t)
         if t is not None and not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    _cuda("workspace", workspace)
+    dev = _one_device(named + (("workspace", workspace),))
     batch, L, H, P = x.shape
     N = B.shape[-1]
     for name, t, shape, dtype in (("x", x, (batch, L, H, P), torch.bfloat16),
@@ -445,8 +493,9 @@ def ssd_fwd(x, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=T
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(int(need), dtype=torch.uint8, device=x.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _abi.check(lib.ssm_scan_fwd_chunked(ctypes.byref(a), _ptr(workspace), ws_bytes,
-                                        _stream(stream)), "ssm_scan_fwd_chunked")
+    with torch.cuda.device(dev):
+        _abi.check(lib.ssm_scan_fwd_chunked(ctypes.byref(a), _ptr(workspace), ws_bytes,
+                                            _stream(stream, dev)), "ssm_scan_fwd_chunked")
     if check_status:
         torch.cuda.synchronize(x.device)
         status = int(workspace[:4].view(torch.int32).item())
