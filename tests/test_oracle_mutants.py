@@ -61,6 +61,54 @@ MUTANTS = [
     ("bwd_softplus_grad", "return s > 20.0 ? 1.0 : 1.0 / (1.0 + exp(-s));",
      "return s > 20.0 ? 1.0 : 1.0 / (1.0 + exp(s));", BWD_PINS),
     ("bwd_gate_grad", "(sg * (1.0 + zv * (1.0 - sg)))", "(sg * (1.0 + zv * sg))", BWD_PINS),
+    # step size: the bias must act with softplus off too, and the cutoff
+    # where softplus(s) is taken as s must sit where the two agree
+    ("softplus_off_drops_bias", "return softplus ? softplus_d(s) : s;",
+     "return softplus ? softplus_d(s) : delta;", ALL_PINS),
+    ("softplus_cutoff_too_low", "return s > 20.0 ? s : log1p(exp(s)); }",
+     "return s > 2.0 ? s : log1p(exp(s)); }", ALL_PINS),
+    # the selective scan: batch and time indexing of the shared and per-row terms
+    ("B_from_batch_0", "const double* Bb = j->B + b * N * L;", "const double* Bb = j->B;",
+     MAMBA1_PINS),
+    ("h0_ignores_batch", "h[n] = j->h0 ? j->h0[row * N + n] : 0.0;",
+     "h[n] = j->h0 ? j->h0[d * N + n] : 0.0;", MAMBA1_PINS),
+    ("skip_uses_previous_u", "(j->D ? j->D[d] * u[t] : 0.0)",
+     "(j->D ? j->D[d] * u[t > 0 ? t - 1 : 0] : 0.0)", MAMBA1_PINS),
+    ("gate_time_shift", "if (j->z) yv *= silu_d(j->z[row * L + t]);",
+     "if (j->z) yv *= silu_d(j->z[row * L + (t > 0 ? t - 1 : 0)]);", MAMBA1_PINS),
+    # the decode step
+    ("step_drop_skip", "double yv = acc + (D ? D[d] * u[row] : 0.0);", "double yv = acc;",
+     MAMBA1_PINS),
+    ("step_drop_gate", "if (z) yv *= silu_d(z[row]);", "if (0) yv *= silu_d(z[row]);",
+     MAMBA1_PINS),
+    ("step_ignores_bias", "step_size(delta[row], bias, d, softplus)",
+     "step_size(delta[row], NULL, d, softplus)", MAMBA1_PINS),
+    # the scalar-decay scan
+    ("ssd_drop_gate", "if (j->z) yv *= silu_d(j->z[xo + p]);",
+     "if (0) yv *= silu_d(j->z[xo + p]);", SSD_PINS),
+    ("ssd_ignores_bias", "step_size(j->delta[(b * L + t) * H + hd], j->bias, hd, j->softplus)",
+     "step_size(j->delta[(b * L + t) * H + hd], NULL, hd, j->softplus)", SSD_PINS),
+    ("ssd_B_time_shift", "const double* Bt = j->B + (b * L + t) * N;",
+     "const double* Bt = j->B + (b * L + (t > 0 ? t - 1 : 0)) * N;", SSD_PINS),
+    ("ssd_x_of_head_0", "const int64_t xo = ((b * L + t) * H + hd) * P;",
+     "const int64_t xo = ((b * L + t) * H) * P;", SSD_PINS),
+    # gradients
+    ("bwd_dC_uses_h_prev", "if (dC) dC[b * N * L + n * L + t] += ds * hs[(t + 1) * N + n];",
+     "if (dC) dC[b * N * L + n * L + t] += ds * hs[t * N + n];", BWD_PINS),
+    ("bwd_dD_ungated", "dDd += ds * ur[t];", "dDd += dy[row * L + t] * ur[t];", BWD_PINS),
+    ("bwd_dB_no_dt", "if (dB) dB[b * N * L + n * L + t] += lam[n] * dt * ur[t];",
+     "if (dB) dB[b * N * L + n * L + t] += lam[n] * ur[t];", BWD_PINS),
+    ("bwd_ddelta_skips_softplus", "const double dd = softplus ? ddt * softplus_grad(sarg) : ddt;",
+     "const double dd = ddt;", BWD_PINS),
+    ("bwd_dz_without_skip", "double sv = D ? D[d] * ur[t] : 0.0;", "double sv = 0.0;", BWD_PINS),
+    ("bwd_adjoint_without_readout", "lam[n] += ds * Cb[n * L + t];", "lam[n] += 0.0 * ds;",
+     BWD_PINS),
+    ("ssd_C_time_shift", "const double* Ct = j->C + (b * L + t) * N;",
+     "const double* Ct = j->C + (b * L + (t > 0 ? t - 1 : 0)) * N;", SSD_PINS),
+    ("ssd_h_last_zero", "j->h_last[row * P * N + i] = S[i];", "j->h_last[row * P * N + i] = 0.0;",
+     SSD_PINS),
+    ("conv_first_tap_only", "for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = 0; k < 1; ++k) {",
+     CONV_PINS),
 ]
 
 
