@@ -38,6 +38,10 @@
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).
  *    Argument checks run on the host before any launch and return
  *    synchronously; a failed launch returns SSM_ERR_CUDA.
+ *  - Kernels launch on the calling thread's current CUDA device: `stream`
+ *    must belong to it, and every device pointer (workspace and staging
+ *    included) must be memory that device can address, normally its own.
+ *    The library cannot check this.
  *  - Outputs must not alias inputs, except `state` of ssm_scan_step.
  *  - Floating-point work is done in fp32; bf16 tensors are widened on load
  *    and y is rounded to nearest-even on store.  The state and h0 / h_last
