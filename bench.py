@@ -18,8 +18,9 @@ bound by its exponentials and fp32 lane operations, not by HBM), the same
 metric end to end through the C ABI from pinned host buffers, clocks sampled
 during the timed region, the CPU oracle as a baseline, and (without --quick)
 one line per other workload: tiny fp32, the 2.8B-layer shape with and
-without gate, the 2^20-step sequence, the Mamba-2 chunked scan and the
-decode step.
+without gate, the 2^20-step sequence, the scan with the convolution stage
+fused in front, the scan's gradients, the Mamba-2 chunked scan, and the
+decode step, eager and replayed from a CUDA graph.
 
 ``--impl reference`` times the CPU oracle instead, on a bounded sample of the
 same workload per step, with the same metric and unit.
@@ -417,6 +418,16 @@ def run_profile(args):
     if args.profile == "scan":
         case = ScanCase(WORKLOAD)
         step = case.step
+    elif args.profile == "bwd":
+        from selective_state_space_08_b200 import api
+        case = ScanCase(WORKLOAD)
+        t = case.t
+        dy = torch.randn(t["u"].shape, dtype=torch.float32, device="cuda")
+        bws = torch.empty(api.scan_bwd_workspace_size(t["u"], t["delta"], t["A"], t["B"], t["C"],
+                                                      t["D"], t["z"], t["delta_bias"], True),
+                          dtype=torch.uint8, device="cuda")
+        step = lambda: api.scan_bwd(t["u"], t["delta"], t["A"], t["B"], t["C"], dy, t["D"],
+                                    t["z"], t["delta_bias"], True, None, workspace=bws)
     else:
         _, step, keep = ssd_case()
     for _ in range(args.warmup + args.steps):
@@ -484,7 +495,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
         "config": describe(c, True) + ", gradients of every input (fp32)",
         "us_per_call": round(sec * 1e6, 2), "GB_per_s": round(bbytes / sec / 1e9, 1),
         "hbm_frac": round(bbytes / sec / 1e9 / hbm_peak, 4),
-        "elems_per_s": round(elems / sec, 1), "launches_per_call": 1}
+        "elems_per_s": round(elems / sec, 1), "launches_per_call": 2}
     del case, dy, bws, bstep
     torch.cuda.empty_cache()
     # Mamba-2 chunked scan (tensor cores)
@@ -658,10 +669,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the other workloads")
-    ap.add_argument("--profile", choices=["scan", "ssd"], default=None,
-                    help="only run the product call of the scan (mamba130m_layer) or\n"
-                         "chunked-scan (mamba2_ssd) workload warmup + steps times,\n"
-                         "untimed, for a profiler to capture")
+    ap.add_argument("--profile", choices=["scan", "bwd", "ssd"], default=None,
+                    help="only run the product call of the scan (mamba130m_layer), its\n"
+                         "gradients (same shape) or the chunked-scan (mamba2_ssd)\n"
+                         "workload warmup + steps times, untimed, for a profiler to capture")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
