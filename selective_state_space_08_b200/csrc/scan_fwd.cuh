@@ -117,10 +117,10 @@ struct alignas(16) BCRows<true> {
 };
 
 // Which rows a variant reads.  Widening packed rows costs 8 integer operations
-// per lane and step: that pays where the shared-memory pipe limits (variants
-// without the gate, 5 blocks per SM; 588 against 620 us on a 4 x 5120 x 4096
-// scan) but not in the gated full pass, whose warps at 3 blocks per SM wait
-// on latency (215 against 207 us on an 8 x 1536 x 2048 scan).
+// per lane and step.  Measured: the variants without the gate gain (578
+// against 620 us on a 4 x 5120 x 4096 scan); the gated full pass does not
+// (215 against 207 us on an 8 x 1536 x 2048 scan, even on the larger one),
+// so it keeps fp32 rows.
 template <typename T, int MODE, bool HAS_Z>
 constexpr bool packed_bc() {
   return std::is_same_v<T, __nv_bfloat16> && !(HAS_Z && MODE == kFull);
