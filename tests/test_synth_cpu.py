@@ -52,11 +52,12 @@ def test_distributions_follow_the_recipe():
     # A = -exp(U(ln 1, ln 10))
     assert inp["A"].max() <= -1.0 and inp["A"].min() >= -10.0
     la = np.log(-inp["A"].astype(np.float64))
-    assert abs(la.mean() - np.log(10) / 2) < 0.02
+    assert abs(la.mean() - np.log(10) / 2) < 5 * np.log(10) / np.sqrt(12 * dim * N)
     # softplus(bias) log-uniform in [1e-3, 1e-1]
     s = np.log1p(np.exp(inp["delta_bias"].astype(np.float64)))
     assert s.min() >= 1e-3 * (1 - 1e-5) and s.max() <= 1e-1 * (1 + 1e-5)
-    assert abs(np.log(s).mean() - (np.log(1e-3) + np.log(1e-1)) / 2) < 0.05
+    width = np.log(1e-1) - np.log(1e-3)   # uniform in log space: sd = width / sqrt(12)
+    assert abs(np.log(s).mean() - (np.log(1e-3) + np.log(1e-1)) / 2) < 5 * width / np.sqrt(12 * dim)
     # the sequence tensors and D are standard normal: mean and standard
     # deviation within 5 standard errors of 0 and 1
     for k in ("u", "delta", "z", "B", "C", "D"):
