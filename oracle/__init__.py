@@ -8,9 +8,13 @@ and this package imports nothing from the library.
 Functions (all take and return numpy arrays; inputs are widened to float64
 exactly, outputs are float64):
 
-* ``scan_fwd``  -- the Mamba-1 selective scan over a whole sequence;
-* ``scan_step`` -- one decode step with the state updated in place;
-* ``ssd_fwd``   -- the Mamba-2 scalar-decay scan, sequential in time.
+* ``scan_fwd``      -- the Mamba-1 selective scan over a whole sequence;
+* ``scan_step``     -- one decode step with the state updated in place;
+* ``ssd_fwd``       -- the Mamba-2 scalar-decay scan, sequential in time;
+* ``conv_silu``     -- the causal depthwise convolution and SiLU in front of
+  the scan;
+* ``scan_fwd_conv`` -- that stage followed by the scan;
+* ``scan_bwd``      -- the gradients of the scan for a given dy.
 
 Each follows the passages cited in ``ssm_oracle.c``.
 """
