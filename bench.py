@@ -559,9 +559,9 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     world, rank, local = dist_env()
+    torch.cuda.set_device(local)  # before the process group, so NCCL binds this rank's GPU
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     hbm_peak, sm_max_mhz, peak_kind = peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
