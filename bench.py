@@ -163,11 +163,22 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self._h = self._handle(pynvml, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:  # noqa: BLE001 -- no NVML: no clock record
             self._nv = None
         self._t = threading.Thread(target=self._run, daemon=True)
+
+    @staticmethod
+    def _handle(nv, index):
+        """NVML handle of CUDA device ``index``, matched by UUID: the CUDA and
+        NVML numberings differ when CUDA_VISIBLE_DEVICES remaps devices."""
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:  # noqa: BLE001 -- fall back to the same index
+            return nv.nvmlDeviceGetHandleByIndex(index)
 
     def _sample(self):
         nv = self._nv
