@@ -297,22 +297,48 @@ class ScanCase:
         api.scan_fwd(*self.args(), y=self.y, h_last=self.h, workspace=self.ws)
 
 
-def time_steps(step, steps, warmup, flush, world, device, sampler_index=None):
+class nvtx_range:
+    """An NVTX range around a block (visible to Nsight tools, e.g. ncu's
+    --nvtx-include); does nothing where NVTX is unavailable."""
+
+    def __init__(self, name):
+        self.name, self.on = name, False
+
+    def __enter__(self):
+        try:
+            import torch
+            torch.cuda.nvtx.range_push(self.name)
+            self.on = True
+        except Exception:  # noqa: BLE001 -- profiling aid only
+            pass
+        return self
+
+    def __exit__(self, *exc):
+        if self.on:
+            try:
+                import torch
+                torch.cuda.nvtx.range_pop()
+            except Exception:  # noqa: BLE001
+                pass
+
+
+def time_steps(step, steps, warmup, flush, world, device, sampler_index=None, name="steps"):
     """W untimed steps, then K steps each bracketed by CUDA events on the
     launching stream, with an L2 flush (outside the events) between them.
     Returns (sum of step times in seconds, max over ranks; per-step ms; clocks)."""
     import torch
     import torch.distributed as dist
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
+    with nvtx_range(f"{name}: warm-up"):
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(sampler_index if sampler_index is not None else 0)
-    with sampler:
+    with sampler, nvtx_range(f"{name}: timed"):
         for k in range(steps):
             flush.zero_()
             starts[k].record()
@@ -455,7 +481,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
                        ("long_seq", True)):
         case = ScanCase(name, gate)
         reps = steps if name != "long_seq" else max(3, min(steps, 10))
-        total, per, _ = time_steps(case.step, reps, min(warmup, 3), flush, 1, None)
+        total, per, _ = time_steps(case.step, reps, min(warmup, 3), flush, 1, None, name=name)
         sec = total / reps
         key = f"{name}{'' if gate else '_nogate'}"
         out[key] = {"config": describe(case.cfg, gate), "us_per_call": round(sec * 1e6, 2),
@@ -475,7 +501,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
     cstep = lambda: api.scan_fwd_conv(t["u"], cw, cb, None, t["delta"], t["A"], t["B"], t["C"],
                                       t["D"], t["z"], t["delta_bias"], True, None, y=case.y,
                                       h_last=case.h, workspace=case.ws)
-    total, per, _ = time_steps(cstep, steps, warmup, flush, 1, None)
+    total, per, _ = time_steps(cstep, steps, warmup, flush, 1, None, name="conv stage")
     sec = total / steps
     cbytes = case.bytes + cw.numel() * 4 + cb.numel() * 4
     out["mamba130m_layer_conv"] = {
@@ -496,7 +522,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
                       dtype=torch.uint8, device="cuda")
     bstep = lambda: api.scan_bwd(t["u"], t["delta"], t["A"], t["B"], t["C"], dy, t["D"], t["z"],
                                  t["delta_bias"], True, None, workspace=bws)
-    total, per, _ = time_steps(bstep, max(3, steps // 4), warmup, flush, 1, None)
+    total, per, _ = time_steps(bstep, max(3, steps // 4), warmup, flush, 1, None, name="gradients")
     sec = total / max(3, steps // 4)
     c = case.cfg
     elems = c["batch"] * c["dim"] * c["seqlen"]
@@ -511,7 +537,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
     torch.cuda.empty_cache()
     # Mamba-2 chunked scan (tensor cores)
     cfg, sstep, keep = ssd_case()
-    total, per, _ = time_steps(sstep, steps, warmup, flush, 1, None)
+    total, per, _ = time_steps(sstep, steps, warmup, flush, 1, None, name="chunked scan")
     sec = total / steps
     sb = ssd_bytes(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"])
     sf = ssd_flops(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"],
@@ -538,7 +564,7 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
             dev(inp["z"][..., 0].copy()), dev(inp["delta_bias"], False)]
     yv = torch.empty((B_, D_), dtype=torch.bfloat16, device="cuda")
     step = lambda: api.scan_step(st, *args, y=yv)
-    total, per, _ = time_steps(step, steps, warmup, flush, 1, None)
+    total, per, _ = time_steps(step, steps, warmup, flush, 1, None, name="decode step")
     sec = total / steps
     sbytes = B_ * D_ * N_ * 8 + B_ * D_ * 2 * 4 + 2 * B_ * N_ * 2 + D_ * (N_ + 2) * 4
     out["decode_step"] = {"config": f"batch={B_} dim={D_} dstate={N_} bf16 gate=on, state fp32",
@@ -556,7 +582,8 @@ def extra_workloads(steps, warmup, flush, hbm_peak):
     with torch.cuda.graph(graph):
         for _ in range(T):
             step()
-    total, per, _ = time_steps(graph.replay, max(3, steps // 8), warmup, flush, 1, None)
+    total, per, _ = time_steps(graph.replay, max(3, steps // 8), warmup, flush, 1, None,
+                               name="decode graph")
     sec = total / max(3, steps // 8) / T
     out["decode_step_graph"] = {"config": f"{out['decode_step']['config']}, {T} steps per graph replay",
                                 "us_per_call": round(sec * 1e6, 3),
@@ -579,7 +606,7 @@ def run_ours(args):
 
     case = ScanCase(WORKLOAD, device=device)
     total, per, clocks = time_steps(case.step, args.steps, args.warmup, flush, world, device,
-                                    sampler_index=local)
+                                    sampler_index=local, name=WORKLOAD)
     sec = total / args.steps
     value = weak_value(case.bytes, world, sec) / 1e9
     elems_s = weak_value(case.elems, world, sec)
